@@ -1,0 +1,225 @@
+"""CRISP sparse prefill on B200: a thin Python binding over libcrisp.so.
+
+Every step of selection and attention runs in the library's CUDA kernels; this module only
+marshals torch tensors (device memory, current stream) into the C ABI declared in
+include/crisp.h. There is no CPU fallback: without the built library (or without a CUDA
+device) every compute call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libcrisp.so")
+
+OK = 0
+STATUS_NAMES = {
+    0: "CRISP_OK", -1: "CRISP_ERR_INVALID_ARG", -2: "CRISP_ERR_UNSUPPORTED", -3: "CRISP_ERR_WORKSPACE",
+    -4: "CRISP_ERR_CUDA", -5: "CRISP_ERR_DEVICE_TIMEOUT", -6: "CRISP_ERR_OVERFLOW", -7: "CRISP_ERR_DEVICE_CHECK",
+}
+EXPORTED = ["crisp_workspace_size", "crisp_select", "crisp_sparse_prefill", "crisp_prefill",
+            "crisp_dense_prefill", "crisp_get_status", "crisp_status_string", "crisp_selftest_timeout"]
+
+
+class CrispError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {STATUS_NAMES.get(code, code)} ({code})")
+        self.code = code
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [("block", ctypes.c_int32), ("anchors", ctypes.c_int32), ("tau_proxy", ctypes.c_float),
+                ("alpha", ctypes.c_float), ("gamma", ctypes.c_float), ("min_blocks", ctypes.c_int32)]
+
+
+class _Index(ctypes.Structure):
+    _fields_ = [("route", ctypes.c_void_p), ("c_struct", ctypes.c_void_p), ("row_ptr", ctypes.c_void_p),
+                ("cols", ctypes.c_void_p), ("debug", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libcrisp.so (built in-tree); raise if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built: run `python -m dynamic_block_sparse_proxy_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        P, I = ctypes.POINTER(_Params), ctypes.POINTER(_Index)
+        L.crisp_workspace_size.argtypes = [i32, i32, i32, i32, P]
+        L.crisp_workspace_size.restype = sz
+        L.crisp_select.argtypes = [vp, vp, i32, i32, i32, i32, P, I, vp, sz, vp]
+        L.crisp_sparse_prefill.argtypes = [vp, vp, vp, i32, i32, i32, i32, I, vp, vp, vp, sz, vp]
+        L.crisp_prefill.argtypes = [vp, vp, vp, i32, i32, i32, i32, P, vp, vp, I, vp, sz, vp]
+        L.crisp_dense_prefill.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, sz, vp]
+        L.crisp_get_status.argtypes = [vp, vp]
+        L.crisp_status_string.argtypes = [i32]
+        L.crisp_status_string.restype = ctypes.c_char_p
+        L.crisp_selftest_timeout.argtypes = [vp, sz, ctypes.c_uint64, vp]
+        for name in ("crisp_select", "crisp_sparse_prefill", "crisp_prefill", "crisp_dense_prefill",
+                     "crisp_get_status", "crisp_selftest_timeout"):
+            getattr(L, name).restype = i32
+        _lib = L
+    return _lib
+
+
+@dataclasses.dataclass
+class Params:
+    """CRISP parameters (paper §3.2, §4, §5). block and anchors must be 128."""
+    block: int = 128
+    anchors: int = 128
+    tau_proxy: float = 0.5
+    alpha: float = 1.0
+    gamma: float = 0.95
+    min_blocks: int = 0
+
+    def c(self) -> _Params:
+        return _Params(self.block, self.anchors, self.tau_proxy, self.alpha, self.gamma, self.min_blocks)
+
+
+@dataclasses.dataclass
+class Index:
+    """Per-head selection result on the device (CSR over query blocks)."""
+    route: torch.Tensor      # int32 [h_q]
+    c_struct: torch.Tensor   # float32 [h_q]
+    row_ptr: torch.Tensor    # int32 [h_q, N_b+1]
+    cols: torch.Tensor       # int32 [h_q, N_b(N_b+1)/2]
+    debug: torch.Tensor | None = None  # float32 [h_q, 2*N_b+4]
+
+    @staticmethod
+    def empty(h_q: int, n: int, device, debug: bool = False) -> "Index":
+        nb = n // 128
+        i32 = dict(device=device, dtype=torch.int32)
+        return Index(torch.empty(h_q, **i32), torch.empty(h_q, device=device, dtype=torch.float32),
+                     torch.empty(h_q, nb + 1, **i32), torch.empty(h_q, nb * (nb + 1) // 2, **i32),
+                     torch.empty(h_q, 2 * nb + 4, device=device, dtype=torch.float32) if debug else None)
+
+    def c(self) -> _Index:
+        return _Index(self.route.data_ptr(), self.c_struct.data_ptr(), self.row_ptr.data_ptr(),
+                      self.cols.data_ptr(), self.debug.data_ptr() if self.debug is not None else None)
+
+    def lists(self, h: int) -> list:
+        """Host copy of head h's per-query-block key-block lists (for inspection and tests)."""
+        rp = self.row_ptr[h].cpu().tolist()
+        cols = self.cols[h].cpu()
+        return [cols[rp[i]:rp[i + 1]].tolist() for i in range(len(rp) - 1)]
+
+
+def _check(code: int, where: str):
+    if code != OK:
+        raise CrispError(code, where)
+
+
+def _stream(t: torch.Tensor) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _qkv_shape(q, k, v=None):
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t is None:
+            continue
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 3:
+            raise ValueError(f"{name} must be a contiguous 3-D bf16 CUDA tensor")
+    h_q, n, d = q.shape
+    h_kv = k.shape[0]
+    if k.shape[1:] != (n, d) or (v is not None and v.shape != k.shape):
+        raise ValueError("q [h_q,n,d], k and v [h_kv,n,d] shapes disagree")
+    return h_q, h_kv, n, d
+
+
+def workspace_size(h_q: int, h_kv: int, n: int, d: int = 128, params: Params | None = None) -> int:
+    p = (params or Params()).c()
+    return int(lib().crisp_workspace_size(h_q, h_kv, n, d, ctypes.byref(p)))
+
+
+def workspace(h_q: int, h_kv: int, n: int, device, d: int = 128) -> torch.Tensor:
+    """Device workspace for this shape, zero-filled (the status word must start at zero)."""
+    nbytes = workspace_size(h_q, h_kv, n, d)
+    if nbytes == 0:
+        raise CrispError(-2, "workspace_size")
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device)
+
+
+def select(q, k, params: Params | None = None, index: Index | None = None, ws: torch.Tensor | None = None,
+           debug: bool = False) -> Index:
+    """Route every q-head and build its key-block lists (crisp_select)."""
+    h_q, h_kv, n, d = _qkv_shape(q, k)
+    params = params or Params()
+    ws = ws if ws is not None else workspace(h_q, h_kv, n, q.device, d)
+    index = index or Index.empty(h_q, n, q.device, debug=debug)
+    p, ix = params.c(), index.c()
+    _check(lib().crisp_select(q.data_ptr(), k.data_ptr(), h_q, h_kv, n, d, ctypes.byref(p), ctypes.byref(ix),
+                              ws.data_ptr(), ws.numel(), _stream(q)), "crisp_select")
+    return index
+
+
+def sparse_prefill(q, k, v, index: Index, o=None, lse=None, ws=None, want_lse: bool = True):
+    """Block-sparse causal attention over `index` (crisp_sparse_prefill). Returns (o, lse)."""
+    h_q, h_kv, n, d = _qkv_shape(q, k, v)
+    ws = ws if ws is not None else workspace(h_q, h_kv, n, q.device, d)
+    o = o if o is not None else torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(h_q, n, device=q.device, dtype=torch.float32)
+    ix = index.c()
+    _check(lib().crisp_sparse_prefill(q.data_ptr(), k.data_ptr(), v.data_ptr(), h_q, h_kv, n, d, ctypes.byref(ix),
+                                      o.data_ptr(), lse.data_ptr() if lse is not None else None, ws.data_ptr(),
+                                      ws.numel(), _stream(q)), "crisp_sparse_prefill")
+    return o, lse
+
+
+def prefill(q, k, v, params: Params | None = None, index: Index | None = None, o=None, lse=None, ws=None,
+            want_lse: bool = True, keep_index: bool = True):
+    """Selection + block-sparse attention (crisp_prefill). Returns (o, lse, index or None)."""
+    h_q, h_kv, n, d = _qkv_shape(q, k, v)
+    params = params or Params()
+    ws = ws if ws is not None else workspace(h_q, h_kv, n, q.device, d)
+    o = o if o is not None else torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(h_q, n, device=q.device, dtype=torch.float32)
+    if index is None and keep_index:
+        index = Index.empty(h_q, n, q.device)
+    p = params.c()
+    ix = ctypes.byref(index.c()) if index is not None else None
+    _check(lib().crisp_prefill(q.data_ptr(), k.data_ptr(), v.data_ptr(), h_q, h_kv, n, d, ctypes.byref(p),
+                               o.data_ptr(), lse.data_ptr() if lse is not None else None, ix, ws.data_ptr(),
+                               ws.numel(), _stream(q)), "crisp_prefill")
+    return o, lse, index
+
+
+def dense_prefill(q, k, v, o=None, lse=None, ws=None, want_lse: bool = True):
+    """Dense causal attention with the same kernel (crisp_dense_prefill). Returns (o, lse)."""
+    h_q, h_kv, n, d = _qkv_shape(q, k, v)
+    ws = ws if ws is not None else workspace(h_q, h_kv, n, q.device, d)
+    o = o if o is not None else torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(h_q, n, device=q.device, dtype=torch.float32)
+    _check(lib().crisp_dense_prefill(q.data_ptr(), k.data_ptr(), v.data_ptr(), h_q, h_kv, n, d, o.data_ptr(),
+                                     lse.data_ptr() if lse is not None else None, ws.data_ptr(), ws.numel(),
+                                     _stream(q)), "crisp_dense_prefill")
+    return o, lse
+
+
+def get_status(ws: torch.Tensor) -> int:
+    """Synchronise the current stream and return (and clear) the device status word."""
+    return int(lib().crisp_get_status(ws.data_ptr(), _stream(ws)))
+
+
+def check_status(ws: torch.Tensor, where: str = "device"):
+    _check(get_status(ws), where)
+
+
+def selftest_timeout(ws: torch.Tensor, limit_ns: int) -> int:
+    """Run the device timeout self-test (a wait nothing satisfies) and return the status it left."""
+    _check(lib().crisp_selftest_timeout(ws.data_ptr(), ws.numel(), limit_ns, _stream(ws)), "crisp_selftest_timeout")
+    return get_status(ws)
+
+
+__all__ = ["Params", "Index", "CrispError", "lib", "workspace_size", "workspace", "select", "sparse_prefill",
+           "prefill", "dense_prefill", "get_status", "check_status", "selftest_timeout", "EXPORTED", "LIB_PATH"]

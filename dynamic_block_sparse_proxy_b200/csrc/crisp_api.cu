@@ -1,0 +1,286 @@
+// crisp_api.cu — the C ABI of libcrisp: argument validation, workspace layout, TMA descriptor
+// encoding and the launch sequence of each entry point. Nothing here allocates device memory;
+// every buffer comes from the caller.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+
+#include "crisp_internal.h"
+#include "sm100.cuh"
+
+namespace crisp {
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  // Resolved once through the runtime (no link-time dependency on libcuda).
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// 2D bf16 view [rows][128] with 64x128 boxes and 128-byte swizzle.
+int make_map(CUtensorMap* m, const void* base, uint64_t rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return CRISP_ERR_CUDA;
+  cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)kB};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? CRISP_OK : CRISP_ERR_CUDA;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_shape(int h_q, int h_kv, int n, int d, Shape* s) {
+  if (h_q <= 0 || h_kv <= 0 || n <= 0 || d <= 0) return CRISP_ERR_INVALID_ARG;
+  if (d != kD || n % kB != 0 || h_q % h_kv != 0) return CRISP_ERR_UNSUPPORTED;
+  const long long nb = n / kB;
+  const long long cap = nb * (nb + 1) / 2;
+  if (cap > 0x7fffffffLL || (long long)h_q * n > 0x7fffffffLL || (long long)h_kv * n > 0x7fffffffLL)
+    return CRISP_ERR_OVERFLOW;
+  s->h_q = h_q;
+  s->h_kv = h_kv;
+  s->n = n;
+  s->nb = (int)nb;
+  s->G = h_q / h_kv;
+  s->n_chunks = (int)((nb + kProxyChunk - 1) / kProxyChunk);
+  s->cap = cap;
+  return CRISP_OK;
+}
+
+int check_params(const crisp_params* p) {
+  if (p == nullptr) return CRISP_ERR_INVALID_ARG;
+  if (p->block != kB || p->anchors != kB) return CRISP_ERR_UNSUPPORTED;
+  if (!std::isfinite(p->tau_proxy) || !std::isfinite(p->alpha) || !std::isfinite(p->gamma))
+    return CRISP_ERR_INVALID_ARG;
+  if (p->alpha < 0.f || p->gamma <= 0.f || p->min_blocks < 0) return CRISP_ERR_INVALID_ARG;
+  return CRISP_OK;
+}
+
+int check_index(const crisp_index* idx, bool need_select_fields) {
+  if (idx == nullptr || idx->row_ptr == nullptr || idx->cols == nullptr) return CRISP_ERR_INVALID_ARG;
+  if (need_select_fields && (idx->route == nullptr || idx->c_struct == nullptr)) return CRISP_ERR_INVALID_ARG;
+  if (!aligned(idx->row_ptr, 4) || !aligned(idx->cols, 4)) return CRISP_ERR_INVALID_ARG;
+  return CRISP_OK;
+}
+
+int check_ws(void* ws, size_t ws_bytes, const Shape& s) {
+  if (ws == nullptr || !aligned(ws, 256)) return CRISP_ERR_INVALID_ARG;
+  if (ws_bytes < workspace_layout(s).total) return CRISP_ERR_WORKSPACE;
+  return CRISP_OK;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+int run_select(const void* q, const void* k, const Shape& s, const crisp_params* p, const crisp_index& out,
+               void* ws, cudaStream_t st) {
+  const Workspace w = workspace_layout(s);
+  SelectArgs a{};
+  a.s = s;
+  a.tau = p->tau_proxy;
+  a.alpha = p->alpha;
+  a.gamma = p->gamma;
+  a.min_blocks = p->min_blocks;
+  a.status = at<int>(ws, w.status);
+  a.trace = at<unsigned long long>(ws, w.trace);
+  a.part = at<float2>(ws, w.part);
+  a.chunk_max = at<float>(ws, w.chunk_max);
+  a.chunk_tot = at<float>(ws, w.chunk_tot);
+  a.row_w = at<float>(ws, w.row_w);
+  a.kbar = at<float>(ws, w.kbar);
+  a.qbar = at<float>(ws, w.qbar);
+  a.pbuf = at<float>(ws, w.pbuf);
+  a.hist_cnt = at<uint32_t>(ws, w.hist_cnt);
+  a.hist_mass = at<double>(ws, w.hist_mass);
+  a.cut = at<CutState>(ws, w.cut);
+  a.keep_v = at<uint8_t>(ws, w.keep_v);
+  a.keep_s = at<uint8_t>(ws, w.keep_s);
+  a.cnt = at<int>(ws, w.cnt);
+  a.eqcnt = at<int>(ws, w.eqcnt);
+  a.eqbase = at<int>(ws, w.eqbase);
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.route = out.route;
+  a.c_struct = out.c_struct;
+  a.row_ptr = out.row_ptr;
+  a.cols = out.cols;
+  a.debug = out.debug;
+
+  CUtensorMap qm, km;
+  int rc = make_map(&qm, q, (uint64_t)s.h_q * s.n);
+  if (rc == CRISP_OK) rc = make_map(&km, k, (uint64_t)s.h_kv * s.n);
+  if (rc != CRISP_OK) return rc;
+
+  // The radix histograms accumulate with atomics: start from zero.
+  if (cudaMemsetAsync(a.hist_cnt, 0, (size_t)s.h_q * kHistBins * 4, st) != cudaSuccess ||
+      cudaMemsetAsync(a.hist_mass, 0, (size_t)s.h_q * kHistBins * 8, st) != cudaSuccess ||
+      cudaMemsetAsync(a.cut, 0, (size_t)s.h_q * sizeof(CutState), st) != cudaSuccess)
+    return CRISP_ERR_CUDA;
+  if (launch_proxy_pass(qm, km, a, st) != cudaSuccess) return CRISP_ERR_CUDA;
+  if (launch_route_threshold(a, st) != cudaSuccess) return CRISP_ERR_CUDA;
+  if (launch_pe(a, st) != cudaSuccess) return CRISP_ERR_CUDA;
+  if (launch_merge(a, st) != cudaSuccess) return CRISP_ERR_CUDA;
+  return CRISP_OK;
+}
+
+int run_attention(const void* q, const void* k, const void* v, const Shape& s, const int32_t* row_ptr,
+                  const int32_t* cols, int dense, void* o, float* lse, void* ws, cudaStream_t st) {
+  const Workspace w = workspace_layout(s);
+  AttnArgs a{};
+  a.s = s;
+  a.dense = dense;
+  a.row_ptr = row_ptr;
+  a.cols = cols;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.status = at<int>(ws, w.status);
+  a.trace = at<unsigned long long>(ws, w.trace);
+  a.scale_log2 = 0.12751743074380045f;  // log2(e) / sqrt(128)
+  CUtensorMap qm, km, vm;
+  int rc = make_map(&qm, q, (uint64_t)s.h_q * s.n);
+  if (rc == CRISP_OK) rc = make_map(&km, k, (uint64_t)s.h_kv * s.n);
+  if (rc == CRISP_OK) rc = make_map(&vm, v, (uint64_t)s.h_kv * s.n);
+  if (rc != CRISP_OK) return rc;
+  return launch_sparse_attn(qm, km, vm, a, st) == cudaSuccess ? CRISP_OK : CRISP_ERR_CUDA;
+}
+
+bool tensors_ok(const void* q, const void* k, const void* v) {
+  return q != nullptr && k != nullptr && (v == nullptr || aligned(v, 16)) && aligned(q, 16) && aligned(k, 16);
+}
+
+// Device-side timeout self-test: waits on a barrier that nothing signals.
+__global__ void timeout_selftest_kernel(int* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    if (!mbar_wait(&bar, 0, nullptr, limit_ns)) record_status(status, CRISP_ERR_DEVICE_TIMEOUT);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_timeout_selftest(int* status, unsigned long long limit_ns, cudaStream_t st) {
+  timeout_selftest_kernel<<<1, 32, 0, st>>>(status, limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace crisp
+
+using namespace crisp;
+
+extern "C" {
+
+size_t crisp_workspace_size(int h_q, int h_kv, int n, int d, const crisp_params* params) {
+  Shape s;
+  if (check_shape(h_q, h_kv, n, d, &s) != CRISP_OK) return 0;
+  if (params != nullptr && check_params(params) != CRISP_OK) return 0;
+  return workspace_layout(s).total;
+}
+
+int crisp_select(const void* q, const void* k, int h_q, int h_kv, int n, int d, const crisp_params* params,
+                 const crisp_index* out, void* ws, size_t ws_bytes, void* stream) {
+  Shape s;
+  int rc = check_shape(h_q, h_kv, n, d, &s);
+  if (rc == CRISP_OK) rc = check_params(params);
+  if (rc == CRISP_OK && !tensors_ok(q, k, nullptr)) rc = CRISP_ERR_INVALID_ARG;
+  if (rc == CRISP_OK) rc = check_index(out, true);
+  if (rc == CRISP_OK) rc = check_ws(ws, ws_bytes, s);
+  if (rc != CRISP_OK) return rc;
+  return run_select(q, k, s, params, *out, ws, static_cast<cudaStream_t>(stream));
+}
+
+int crisp_sparse_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv, int n, int d,
+                         const crisp_index* idx, void* o, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  Shape s;
+  int rc = check_shape(h_q, h_kv, n, d, &s);
+  if (rc == CRISP_OK && (!tensors_ok(q, k, v) || v == nullptr || o == nullptr || !aligned(o, 16)))
+    rc = CRISP_ERR_INVALID_ARG;
+  if (rc == CRISP_OK) rc = check_index(idx, false);
+  if (rc == CRISP_OK) rc = check_ws(ws, ws_bytes, s);
+  if (rc != CRISP_OK) return rc;
+  return run_attention(q, k, v, s, idx->row_ptr, idx->cols, 0, o, lse, ws, static_cast<cudaStream_t>(stream));
+}
+
+int crisp_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv, int n, int d,
+                  const crisp_params* params, void* o, float* lse, const crisp_index* idx_out, void* ws,
+                  size_t ws_bytes, void* stream) {
+  Shape s;
+  int rc = check_shape(h_q, h_kv, n, d, &s);
+  if (rc == CRISP_OK) rc = check_params(params);
+  if (rc == CRISP_OK && (!tensors_ok(q, k, v) || v == nullptr || o == nullptr || !aligned(o, 16)))
+    rc = CRISP_ERR_INVALID_ARG;
+  if (rc == CRISP_OK && idx_out != nullptr) rc = check_index(idx_out, true);
+  if (rc == CRISP_OK) rc = check_ws(ws, ws_bytes, s);
+  if (rc != CRISP_OK) return rc;
+  crisp_index idx;
+  if (idx_out != nullptr) {
+    idx = *idx_out;
+  } else {
+    const Workspace w = workspace_layout(s);
+    idx.route = at<int32_t>(ws, w.idx_route);
+    idx.c_struct = at<float>(ws, w.idx_c);
+    idx.row_ptr = at<int32_t>(ws, w.idx_row_ptr);
+    idx.cols = at<int32_t>(ws, w.idx_cols);
+    idx.debug = nullptr;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  rc = run_select(q, k, s, params, idx, ws, st);
+  if (rc != CRISP_OK) return rc;
+  return run_attention(q, k, v, s, idx.row_ptr, idx.cols, 0, o, lse, ws, st);
+}
+
+int crisp_dense_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv, int n, int d, void* o,
+                        float* lse, void* ws, size_t ws_bytes, void* stream) {
+  Shape s;
+  int rc = check_shape(h_q, h_kv, n, d, &s);
+  if (rc == CRISP_OK && (!tensors_ok(q, k, v) || v == nullptr || o == nullptr || !aligned(o, 16)))
+    rc = CRISP_ERR_INVALID_ARG;
+  if (rc == CRISP_OK) rc = check_ws(ws, ws_bytes, s);
+  if (rc != CRISP_OK) return rc;
+  return run_attention(q, k, v, s, nullptr, nullptr, 1, o, lse, ws, static_cast<cudaStream_t>(stream));
+}
+
+int crisp_get_status(void* ws, void* stream) {
+  if (ws == nullptr || !aligned(ws, 256)) return CRISP_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return CRISP_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return CRISP_ERR_CUDA;
+  if (v != 0 && cudaMemset(ws, 0, sizeof(int)) != cudaSuccess) return CRISP_ERR_CUDA;
+  return v;
+}
+
+const char* crisp_status_string(int status) {
+  switch (status) {
+    case CRISP_OK: return "CRISP_OK";
+    case CRISP_ERR_INVALID_ARG: return "CRISP_ERR_INVALID_ARG";
+    case CRISP_ERR_UNSUPPORTED: return "CRISP_ERR_UNSUPPORTED";
+    case CRISP_ERR_WORKSPACE: return "CRISP_ERR_WORKSPACE";
+    case CRISP_ERR_CUDA: return "CRISP_ERR_CUDA";
+    case CRISP_ERR_DEVICE_TIMEOUT: return "CRISP_ERR_DEVICE_TIMEOUT";
+    case CRISP_ERR_OVERFLOW: return "CRISP_ERR_OVERFLOW";
+    case CRISP_ERR_DEVICE_CHECK: return "CRISP_ERR_DEVICE_CHECK";
+    default: return "CRISP_ERR_UNKNOWN";
+  }
+}
+
+int crisp_selftest_timeout(void* ws, size_t ws_bytes, uint64_t limit_ns, void* stream) {
+  if (ws == nullptr || !aligned(ws, 256) || ws_bytes < 256) return CRISP_ERR_INVALID_ARG;
+  return launch_timeout_selftest(static_cast<int*>(ws), limit_ns, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? CRISP_OK
+             : CRISP_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,130 @@
+// crisp_internal.h — shapes, workspace layout and kernel launch declarations shared by the
+// host entry points and the kernels of libcrisp.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "crisp.h"
+
+namespace crisp {
+
+constexpr int kB = 128;        // block size (queries and keys)
+constexpr int kD = 128;        // head dimension
+constexpr int kProxyChunk = 16;  // key blocks per proxy CTA
+constexpr int kHistBins = 2048;  // radix-select bins per pass (11, 10, 10 bits)
+
+struct Shape {
+  int h_q, h_kv, n, nb, G, n_chunks;
+  long long cap;  // per-head capacity of the column array: nb*(nb+1)/2
+};
+
+// State of the Pooled-Estimation cut of one head (device memory, inside the workspace).
+struct CutState {
+  double target;       // gamma * N_b
+  double mass_above;   // mass of entries above the current bucket prefix
+  uint32_t prefix;     // bit prefix fixed so far
+  uint32_t keep_all;   // 1: gamma >= 1 or the target is not reachable -> keep every entry
+  uint32_t thr_bits;   // final threshold value (fp32 bit pattern)
+  uint32_t t_eq;       // entries equal to the threshold to keep, in (qb, kb) order
+  uint32_t count_eq;   // entries equal to the threshold
+  uint32_t pad;
+};
+
+struct Workspace {
+  size_t status, trace, part, chunk_max, chunk_tot, row_w, kbar, qbar, pbuf, hist_cnt, hist_mass, cut,
+      keep_v, keep_s, cnt, eqcnt, eqbase, idx_route, idx_c, idx_row_ptr, idx_cols, total;
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline Workspace workspace_layout(const Shape& s) {
+  Workspace w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  const size_t hq = s.h_q, nb = s.nb, ch = s.n_chunks;
+  w.status = take(256);
+  w.trace = take((size_t)256 * 2 * 8 * 8);
+  w.part = take(hq * nb * kB * 8);
+  w.chunk_max = take(hq * ch * kB * 4);
+  w.chunk_tot = take(hq * ch * kB * 4);
+  w.row_w = take(hq * ch * kB * 4);
+  w.kbar = take((size_t)s.h_kv * nb * kD * 4);
+  w.qbar = take(hq * nb * kD * 4);
+  w.pbuf = take(hq * (size_t)s.cap * 4);
+  w.hist_cnt = take(hq * kHistBins * 4);
+  w.hist_mass = take(hq * kHistBins * 8);
+  w.cut = take(hq * sizeof(CutState));
+  w.keep_v = take(hq * nb);
+  w.keep_s = take(hq * nb);
+  w.cnt = take(hq * nb * 4);
+  w.eqcnt = take(hq * nb * 4);
+  w.eqbase = take(hq * (nb + 1) * 4);
+  w.idx_route = take(hq * 4);
+  w.idx_c = take(hq * 4);
+  w.idx_row_ptr = take(hq * (nb + 1) * 4);
+  w.idx_cols = take(hq * (size_t)s.cap * 4);
+  w.total = off;
+  return w;
+}
+
+// Kernel parameter block for the selection kernels.
+struct SelectArgs {
+  Shape s;
+  float tau, alpha, gamma;
+  int min_blocks;
+  int* status;
+  unsigned long long* trace;
+  float2* part;
+  float* chunk_max;
+  float* chunk_tot;
+  float* row_w;
+  float* kbar;
+  float* qbar;
+  float* pbuf;
+  uint32_t* hist_cnt;
+  double* hist_mass;
+  CutState* cut;
+  uint8_t* keep_v;
+  uint8_t* keep_s;
+  int* cnt;
+  int* eqcnt;
+  int* eqbase;
+  const __nv_bfloat16* q;
+  int32_t* route;
+  float* c_struct;
+  int32_t* row_ptr;
+  int32_t* cols;
+  float* debug;
+};
+
+struct AttnArgs {
+  Shape s;
+  int dense;             // 1: every block <= qb, index ignored
+  const int32_t* row_ptr;
+  const int32_t* cols;
+  __nv_bfloat16* o;
+  float* lse;
+  int* status;
+  unsigned long long* trace;
+  float scale_log2;      // log2(e)/sqrt(d)
+};
+
+// Launchers (return cudaGetLastError()).
+cudaError_t launch_proxy_pass(const CUtensorMap& q_map, const CUtensorMap& k_map, const SelectArgs& a,
+                              cudaStream_t st);
+cudaError_t launch_route_threshold(const SelectArgs& a, cudaStream_t st);
+cudaError_t launch_pe(const SelectArgs& a, cudaStream_t st);
+cudaError_t launch_merge(const SelectArgs& a, cudaStream_t st);
+cudaError_t launch_sparse_attn(const CUtensorMap& q_map, const CUtensorMap& k_map,
+                               const CUtensorMap& v_map, const AttnArgs& a, cudaStream_t st);
+cudaError_t launch_timeout_selftest(int* status, unsigned long long limit_ns, cudaStream_t st);
+
+}  // namespace crisp

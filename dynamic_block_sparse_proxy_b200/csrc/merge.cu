@@ -1,0 +1,220 @@
+// merge.cu — per-query-block key-block lists (CSR) from the routing decisions.
+//
+// Vertical-Slash head, query block qb (CRISP §4: both directions thresholded separately and
+// unioned; the first and last blocks always retained): key block kb <= qb is selected iff
+//   kb == 0, or kb is a kept vertical block (or the last block), or a kept slash offset block m
+//   (or the anchor offsets 0 and N_b-1) satisfies m == qb-kb or m == qb-kb-1.
+// A query in block qb and a key at token offset o in [mB, mB+B) meet in key block qb-m or
+// qb-m-1, so selecting both covers every token of a kept diagonal band.
+// Pooled-Estimation head: (qb, kb) is selected iff its pooled score lies above the cut value T,
+// or equals T and is among the first t_eq such entries in (qb, kb) order, or kb is one of the
+// anchors {0, qb-1, qb}. With N_b <= 2 every causal block is selected.
+//
+// Passes: ties with the cut value per row and their exclusive scan (global tie ranks), the exact
+// count per row and its exclusive scan (row_ptr), then compaction.
+#include "crisp_internal.h"
+#include "sm100.cuh"
+
+namespace crisp {
+namespace {
+
+constexpr int T = 128;
+
+struct RowCtx {
+  int vs, nb, qb;
+  const uint8_t* kv;
+  const uint8_t* ks;
+  const float* P;
+  uint32_t thr;
+  uint32_t keep_all;
+};
+
+__device__ __forceinline__ bool vs_sel(const RowCtx& c, int kb) {
+  if (c.nb <= 2 || kb == 0 || kb == c.nb - 1) return true;
+  if (c.kv[kb]) return true;
+  const int m0 = c.qb - kb;  // offset block m with qb-m == kb
+  if (m0 == 0 || m0 == c.nb - 1 || c.ks[m0]) return true;
+  const int m1 = m0 - 1;     // offset block m with qb-m-1 == kb
+  if (m1 >= 0 && (m1 == 0 || m1 == c.nb - 1 || c.ks[m1])) return true;
+  return false;
+}
+
+// PE: where an entry stands relative to the cut value: 0 below, 1 above, 2 equal. Anchors do not
+// change this: the cut is taken over every entry, and the anchors are added on top.
+__device__ __forceinline__ int pe_cut_flag(const RowCtx& c, int kb) {
+  if (c.keep_all) return 1;
+  const uint32_t bits = __float_as_uint(c.P[kb]);
+  if (bits > c.thr) return 1;
+  return bits == c.thr ? 2 : 0;
+}
+
+__device__ __forceinline__ bool pe_anchor(const RowCtx& c, int kb) {
+  return kb == 0 || kb == c.qb || kb == c.qb - 1;
+}
+
+__device__ __forceinline__ RowCtx make_ctx(const SelectArgs& a, int h, int qb) {
+  RowCtx c;
+  const Shape& s = a.s;
+  c.vs = a.route[h];
+  c.nb = s.nb;
+  c.qb = qb;
+  c.kv = a.keep_v + (size_t)h * s.nb;
+  c.ks = a.keep_s + (size_t)h * s.nb;
+  c.P = a.pbuf + (size_t)h * s.cap + (size_t)qb * (qb + 1) / 2;
+  const CutState cs = a.cut[h];
+  c.thr = cs.thr_bits;
+  c.keep_all = (s.nb <= 2 || c.vs) ? 1u : cs.keep_all;
+  return c;
+}
+
+__device__ __forceinline__ long long tie_quota(const SelectArgs& a, int h) {
+  const CutState cs = a.cut[h];
+  return (a.route[h] || a.s.nb <= 2 || cs.keep_all) ? 0 : (long long)cs.t_eq;
+}
+
+// Block-wide exclusive scan of a 0/1 flag over 128 threads; returns the prefix, total in *tot.
+__device__ __forceinline__ int scan128(int flag, int* wsum, int* tot) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const unsigned bal = __ballot_sync(0xffffffffu, flag);
+  const int pre = __popc(bal & ((1u << lane) - 1u));
+  __syncthreads();
+  if (lane == 0) wsum[w] = __popc(bal);
+  __syncthreads();
+  int off = 0, t = 0;
+#pragma unroll
+  for (int i = 0; i < T / 32; ++i) {
+    if (i < w) off += wsum[i];
+    t += wsum[i];
+  }
+  *tot = t;
+  return off + pre;
+}
+
+// Walks row qb of head h in key-block order and calls emit(kb) for every selected block.
+// Entries tied with the cut value are ranked over the whole head in (qb, kb) order, starting
+// from eqbase[qb]; the first t_eq of them are kept.
+template <typename Emit>
+__device__ __forceinline__ int walk_row(const SelectArgs& a, int h, int qb, long long erank, Emit emit) {
+  const RowCtx c = make_ctx(a, h, qb);
+  const bool vsrow = c.vs || a.s.nb <= 2;
+  const long long t_eq = tie_quota(a, h);
+  __shared__ int wsum[T / 32];
+  int count = 0;
+  for (int base = 0; base <= qb; base += T) {
+    const int kb = base + threadIdx.x;
+    int sel = 0, eqf = 0;
+    if (kb <= qb) {
+      if (vsrow) {
+        sel = vs_sel(c, kb);
+      } else {
+        const int f = pe_cut_flag(c, kb);
+        sel = (f == 1) || pe_anchor(c, kb);
+        eqf = f == 2;
+      }
+    }
+    if (!vsrow) {
+      int etot;
+      const int epre = scan128(eqf, wsum, &etot);
+      if (eqf && erank + epre < t_eq) sel = 1;
+      erank += etot;
+    }
+    int stot;
+    const int spre = scan128(sel, wsum, &stot);
+    if (sel) emit(kb, count + spre);
+    count += stot;
+  }
+  return count;
+}
+
+// Pass 1: entries of each PE row that tie with the cut value.
+__global__ void __launch_bounds__(T) merge_ties_kernel(const SelectArgs a) {
+  const int qb = blockIdx.x, h = blockIdx.y;
+  const RowCtx c = make_ctx(a, h, qb);
+  int ne = 0;
+  if (!(c.vs || a.s.nb <= 2))
+    for (int kb = threadIdx.x; kb <= qb; kb += T) ne += pe_cut_flag(c, kb) == 2;
+  __shared__ int red[T / 32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ne += __shfl_xor_sync(0xffffffffu, ne, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ne;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int t = 0;
+    for (int i = 0; i < T / 32; ++i) t += red[i];
+    a.eqcnt[(size_t)h * a.s.nb + qb] = t;
+  }
+}
+
+// Pass 2: exact number of selected blocks per row.
+__global__ void __launch_bounds__(T) merge_count_kernel(const SelectArgs a) {
+  const int qb = blockIdx.x, h = blockIdx.y;
+  const long long erank = a.eqbase[(size_t)h * (a.s.nb + 1) + qb];
+  const int n = walk_row(a, h, qb, erank, [](int, int) {});
+  if (threadIdx.x == 0) a.cnt[(size_t)h * a.s.nb + qb] = n;
+}
+
+// Pass 3: compaction into the CSR column array.
+__global__ void __launch_bounds__(T) merge_write_kernel(const SelectArgs a) {
+  const int qb = blockIdx.x, h = blockIdx.y;
+  const int nb = a.s.nb;
+  const long long erank = a.eqbase[(size_t)h * (nb + 1) + qb];
+  int32_t* out = a.cols + (size_t)h * a.s.cap + a.row_ptr[(size_t)h * (nb + 1) + qb];
+  walk_row(a, h, qb, erank, [out](int kb, int pos) { out[pos] = kb; });
+}
+
+// One CTA per head: exclusive scan of in[h][0..nb) into out[h][0..nb] (out[nb] = total).
+__global__ void __launch_bounds__(1024) scan_rows_kernel(const int* in, int* out, int nb, float* debug_total) {
+  const int h = blockIdx.x;
+  const int* src = in + (size_t)h * nb;
+  int* dst = out + (size_t)h * (nb + 1);
+  __shared__ int wsum[32];
+  __shared__ long long carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  for (int base = 0; base < nb; base += 1024) {
+    const int i = base + threadIdx.x;
+    const int v = i < nb ? src[i] : 0;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[w] = x;
+    __syncthreads();
+    if (w == 0) {
+      int t = wsum[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, t, o);
+        if (lane >= o) t += y;
+      }
+      wsum[lane] = t;
+    }
+    __syncthreads();
+    const long long before = carry + (w > 0 ? wsum[w - 1] : 0) + x - v;
+    if (i < nb) dst[i] = (int)before;
+    __syncthreads();
+    if (threadIdx.x == 0) carry += wsum[31];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    dst[nb] = (int)carry;
+    if (debug_total != nullptr) debug_total[(size_t)h * (2 * nb + 4) + 2 * nb + 3] = (float)carry;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_merge(const SelectArgs& a, cudaStream_t st) {
+  const Shape& s = a.s;
+  merge_ties_kernel<<<dim3(s.nb, s.h_q), T, 0, st>>>(a);
+  scan_rows_kernel<<<s.h_q, 1024, 0, st>>>(a.eqcnt, a.eqbase, s.nb, nullptr);
+  merge_count_kernel<<<dim3(s.nb, s.h_q), T, 0, st>>>(a);
+  scan_rows_kernel<<<s.h_q, 1024, 0, st>>>(a.cnt, a.row_ptr, s.nb, a.debug);
+  merge_write_kernel<<<dim3(s.nb, s.h_q), T, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace crisp

@@ -1,0 +1,148 @@
+/*
+ * crisp.h — C ABI of the CRISP sparse-prefill library (libcrisp.so) for NVIDIA B200 (sm_100a).
+ *
+ * The library computes the prefill hot path of CRISP ("CRISP: Cliff-awaRe Input-adaptive Sparse
+ * Prefilling with Structural-Mass-Motivated Routing"): per-head index selection from a proxy
+ * attention over the last query block, then causal attention restricted to the selected
+ * (query block, key block) pairs.
+ *
+ * Conventions shared by every entry point
+ *   - Q is bf16 [h_q][n][d], K and V are bf16 [h_kv][n][d], all contiguous, in device memory.
+ *     GQA: q-head h reads kv-head h / (h_q / h_kv) (consecutive q-heads share a kv-head).
+ *   - Supported shapes: d == 128, block == 128, anchors == 128, n a multiple of 128, n >= 128,
+ *     h_q a multiple of h_kv. Anything else returns CRISP_ERR_UNSUPPORTED before any launch.
+ *   - N_b = n / 128 is the number of blocks.
+ *   - Ownership: the caller allocates every buffer (inputs, outputs, index, workspace); the
+ *     library never allocates or frees memory and keeps no global mutable state. Calls on
+ *     different streams are safe when each uses its own workspace.
+ *   - All compute calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream). They return CRISP_OK once the work is enqueued. Errors found on the host are
+ *     returned directly and nothing is launched; errors found on the device (a bounded wait
+ *     that ran out, a failed self-check) are recorded in the workspace's status word and read
+ *     with crisp_get_status().
+ *   - Pointers must be 16-byte aligned (TMA requirement); the workspace 256-byte aligned.
+ *   - The workspace's first 256 bytes hold the device status word: zero them once after
+ *     allocating the workspace (e.g. cudaMemset); crisp_get_status() clears it after reading.
+ *     The rest of the workspace needs no initialisation and may hold anything between calls.
+ */
+#ifndef CRISP_H
+#define CRISP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes: 0 is success, negative values are errors. */
+enum {
+  CRISP_OK = 0,
+  CRISP_ERR_INVALID_ARG = -1,    /* null pointer, bad parameter value, misaligned pointer */
+  CRISP_ERR_UNSUPPORTED = -2,    /* shape outside the supported set (see above) */
+  CRISP_ERR_WORKSPACE = -3,      /* ws_bytes < crisp_workspace_size(...) */
+  CRISP_ERR_CUDA = -4,           /* a CUDA runtime/driver call or a launch failed */
+  CRISP_ERR_DEVICE_TIMEOUT = -5, /* a device-side wait exceeded its limit; the kernel exited */
+  CRISP_ERR_OVERFLOW = -6,       /* sizes overflow the 32-bit index formats */
+  CRISP_ERR_DEVICE_CHECK = -7    /* a device-side consistency check failed */
+};
+
+/*
+ * Method parameters (CRISP paper §3.2, §4, §5; the per-head pseudocode of the rcap.io summary).
+ *   block      query/key block size B (must be 128)
+ *   anchors    sink window (first `anchors` keys) and recency window (last `anchors` keys) of
+ *              the C_struct routing signal (must be 128)
+ *   tau_proxy  route a head to Vertical-Slash iff C_struct >= tau_proxy
+ *   alpha      Vertical-Slash keep rule: block j kept iff p[j] > alpha * mu (alpha >= 0)
+ *   gamma      Pooled-Estimation coverage target of the global cumulative cut (gamma > 0;
+ *              gamma >= 1 keeps every causal block)
+ *   min_blocks minimum kept blocks per direction on Vertical-Slash heads (>= 0; 0 = off)
+ */
+typedef struct {
+  int32_t block;
+  int32_t anchors;
+  float tau_proxy;
+  float alpha;
+  float gamma;
+  int32_t min_blocks;
+} crisp_params;
+
+/*
+ * Per-head index sets in CSR form, written by crisp_select / crisp_prefill and read by
+ * crisp_sparse_prefill. All arrays are device memory owned by the caller.
+ *   route    int32 [h_q]        1 = Vertical-Slash, 0 = Pooled-Estimation
+ *   c_struct float [h_q]        C_struct of each head (CRISP §3.2)
+ *   row_ptr  int32 [h_q][N_b+1] row qb of head h spans cols[h*cap + row_ptr[h][qb] ..
+ *                               h*cap + row_ptr[h][qb+1]), cap = N_b*(N_b+1)/2
+ *   cols     int32 [h_q][cap]   key-block indices, strictly ascending within a row, each <= qb
+ *   debug    float [h_q][2*N_b+4] or NULL: p_v[N_b], p_s[N_b] (vertical and slash block
+ *            masses, CRISP §4), then mu_v, mu_s, C_struct, and the number of selected pairs
+ */
+typedef struct {
+  int32_t* route;
+  float* c_struct;
+  int32_t* row_ptr;
+  int32_t* cols;
+  float* debug;
+} crisp_index;
+
+/* Bytes of device workspace needed by every compute call for this shape (0 if unsupported). */
+size_t crisp_workspace_size(int h_q, int h_kv, int n, int d, const crisp_params* params);
+
+/*
+ * Index selection (CRISP §2 proxy attention over the last query block; §3.2 C_struct routing;
+ * §4 vertical/slash block pooling, noise floor mu = max(1-p[0]-p[-1],0)/(N_b-2), keep p[j] >
+ * alpha*mu, union of both directions; Pooled-Estimation: pooled Q/K block scores, softmax,
+ * global gamma cumulative cut). Writes every field of *out (debug if non-NULL).
+ */
+int crisp_select(const void* q, const void* k, int h_q, int h_kv, int n, int d,
+                 const crisp_params* params, const crisp_index* out,
+                 void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Block-sparse causal attention (CRISP §2: softmax(QK^T/sqrt(d) + M_S) V with M_S = 0 on the
+ * selected blocks and -inf elsewhere; within a block, key j is visible to query i iff j <= i).
+ * Reads idx->row_ptr and idx->cols; every row must contain at least one block <= qb.
+ * o: bf16 [h_q][n][d]. lse: fp32 [h_q][n] natural-log sum-exp of the scaled logits, or NULL.
+ */
+int crisp_sparse_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv, int n,
+                         int d, const crisp_index* idx, void* o, float* lse,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Selection followed by block-sparse attention in one call. idx_out may be NULL, in which
+ * case the index lives inside the workspace; otherwise it receives the index as crisp_select.
+ */
+int crisp_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv, int n, int d,
+                  const crisp_params* params, void* o, float* lse, const crisp_index* idx_out,
+                  void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Dense causal attention with the same kernel (every block <= qb selected): the reference
+ * point for the sparse-versus-dense speed ratio. Same buffers as crisp_sparse_prefill.
+ */
+int crisp_dense_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv, int n,
+                        int d, void* o, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, returns the device status word of `ws` (CRISP_OK or the first device
+ * error recorded since the last call) and clears it. Returns CRISP_ERR_CUDA if the
+ * synchronisation itself fails.
+ */
+int crisp_get_status(void* ws, void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* crisp_status_string(int status);
+
+/*
+ * Self-test of the device-side timeout path: launches one block that waits on a barrier
+ * nothing signals, with a wait limit of `limit_ns` nanoseconds; the kernel then records
+ * CRISP_ERR_DEVICE_TIMEOUT in the status word and exits. Nothing faults or hangs.
+ */
+int crisp_selftest_timeout(void* ws, size_t ws_bytes, uint64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CRISP_H */

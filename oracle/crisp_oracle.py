@@ -241,22 +241,26 @@ def select_head(q: np.ndarray, k: np.ndarray, *, block=128, anchors=128, tau_pro
 # ----------------------------------------------------------------------------------------------
 # Attention on an index set  ([CRISP] §2: softmax(QK^T/sqrt(d) + M_S) V)
 # ----------------------------------------------------------------------------------------------
-def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, key_blocks, qb: int, B: int = 128):
-    """Output rows of query block qb attending to the keys of `key_blocks`, causally.
-
-    O[i] = sum_{j in S(qb), j <= i} softmax_j(q_i . k_j / sqrt(d)) v_j, fp64.
+def attention_block(q_blk: np.ndarray, k: np.ndarray, v: np.ndarray, key_blocks, qb: int, B: int = 128):
+    """Output rows of query block qb (queries q_blk = q[qb*B:(qb+1)*B]) attending to the keys of
+    `key_blocks`, causally: O[i] = sum_{j in S(qb), j <= i} softmax_j(q_i . k_j / sqrt(d)) v_j.
     Returns (O [B, d], lse [B]) with lse the natural-log sum of exp of the scaled logits.
     """
-    d = q.shape[1]
+    d = q_blk.shape[1]
     keys = np.concatenate([np.arange(kb * B, kb * B + B) for kb in key_blocks])
     rows = np.arange(qb * B, qb * B + B)
-    s = (q[rows] @ k[keys].T) / np.sqrt(d)
+    s = (q_blk @ k[keys].T) / np.sqrt(d)
     allowed = keys[None, :] <= rows[:, None]
     s = np.where(allowed, s, -np.inf)
     m = s.max(axis=1, keepdims=True)
     e = np.where(allowed, np.exp(s - m), 0.0)
     z = e.sum(axis=1, keepdims=True)
     return (e / z) @ v[keys], (m + np.log(z))[:, 0]
+
+
+def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, key_blocks, qb: int, B: int = 128):
+    """attention_block for query block qb of a full query matrix q [n, d]."""
+    return attention_block(q[qb * B:(qb + 1) * B], k, v, key_blocks, qb, B)
 
 
 def attention_head(q, k, v, lists, B: int = 128):

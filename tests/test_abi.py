@@ -1,0 +1,116 @@
+"""C-ABI checks that need no GPU: the library loads, exports every declared entry point, sizes
+its workspace, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import dynamic_block_sparse_proxy_b200 as crisp
+from dynamic_block_sparse_proxy_b200 import build as B
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "crisp.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return crisp.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(crisp_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_names():
+    assert declared_functions() == sorted(crisp.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for code, name in crisp.STATUS_NAMES.items():
+        assert L.crisp_status_string(code).decode() == name
+    assert L.crisp_status_string(12345).decode() == "CRISP_ERR_UNKNOWN"
+
+
+def test_workspace_size(L):
+    p = crisp.Params().c()
+    small = L.crisp_workspace_size(1, 1, 4096, 128, ctypes.byref(p))
+    big = L.crisp_workspace_size(32, 8, 131072, 128, ctypes.byref(p))
+    assert 0 < small < big
+    # dominated by the per-head pooled-score and column arrays: 2 * 4 B * h_q * N_b(N_b+1)/2
+    nb = 131072 // 128
+    assert big > 8 * 32 * nb * (nb + 1) // 2
+    assert big % 256 == 0
+    for bad in [(1, 1, 4096, 64), (1, 1, 4000, 128), (3, 2, 4096, 128), (0, 1, 4096, 128), (1, 1, 0, 128)]:
+        assert L.crisp_workspace_size(*bad, ctypes.byref(p)) == 0
+    q = crisp.Params(block=64).c()
+    assert L.crisp_workspace_size(1, 1, 4096, 128, ctypes.byref(q)) == 0
+
+
+def _idx(route=1, c=1, rp=1, cols=1):
+    return crisp._Index(0x1000 if route else None, 0x1000 if c else None, 0x1000 if rp else None,
+                        0x1000 if cols else None, None)
+
+
+def test_select_rejects_bad_arguments_before_launch(L):
+    p = crisp.Params().c()
+    ws = 0x100000
+    big = 1 << 40
+    fake = 0x10000
+    ix = _idx()
+    cases = [
+        ((None, fake, 1, 1, 4096, 128, ctypes.byref(p), ctypes.byref(ix), ws, big, None), crisp.STATUS_NAMES[-1]),
+        ((fake, fake, 1, 1, 4096, 64, ctypes.byref(p), ctypes.byref(ix), ws, big, None), crisp.STATUS_NAMES[-2]),
+        ((fake, fake, 1, 1, 4000, 128, ctypes.byref(p), ctypes.byref(ix), ws, big, None), crisp.STATUS_NAMES[-2]),
+        ((fake, fake, 3, 2, 4096, 128, ctypes.byref(p), ctypes.byref(ix), ws, big, None), crisp.STATUS_NAMES[-2]),
+        ((fake, fake, 1, 1, 4096, 128, None, ctypes.byref(ix), ws, big, None), crisp.STATUS_NAMES[-1]),
+        ((fake, fake, 1, 1, 4096, 128, ctypes.byref(p), None, ws, big, None), crisp.STATUS_NAMES[-1]),
+        ((fake, fake, 1, 1, 4096, 128, ctypes.byref(p), ctypes.byref(_idx(rp=0)), ws, big, None), crisp.STATUS_NAMES[-1]),
+        ((fake, fake, 1, 1, 4096, 128, ctypes.byref(p), ctypes.byref(ix), ws, 1024, None), crisp.STATUS_NAMES[-3]),
+        ((fake, fake, 1, 1, 4096, 128, ctypes.byref(p), ctypes.byref(ix), ws + 8, big, None), crisp.STATUS_NAMES[-1]),
+        ((fake + 2, fake, 1, 1, 4096, 128, ctypes.byref(p), ctypes.byref(ix), ws, big, None), crisp.STATUS_NAMES[-1]),
+    ]
+    for args, want in cases:
+        assert crisp.STATUS_NAMES[L.crisp_select(*args)] == want, args
+    for bad in (crisp.Params(alpha=-1.0), crisp.Params(gamma=0.0), crisp.Params(min_blocks=-1),
+                crisp.Params(tau_proxy=float("nan")), crisp.Params(anchors=64)):
+        bp = bad.c()
+        rc = L.crisp_select(fake, fake, 1, 1, 4096, 128, ctypes.byref(bp), ctypes.byref(ix), ws, big, None)
+        assert rc in (-1, -2), bad
+
+
+def test_attention_entry_points_reject_bad_arguments(L):
+    fake, ws, big = 0x10000, 0x100000, 1 << 40
+    ix = _idx()
+    assert L.crisp_sparse_prefill(fake, fake, None, 1, 1, 4096, 128, ctypes.byref(ix), fake, None, ws, big, None) == -1
+    assert L.crisp_sparse_prefill(fake, fake, fake, 1, 1, 4096, 128, ctypes.byref(_idx(cols=0)), fake, None, ws, big,
+                                  None) == -1
+    assert L.crisp_sparse_prefill(fake, fake, fake, 1, 1, 4096, 128, ctypes.byref(ix), None, None, ws, big, None) == -1
+    assert L.crisp_sparse_prefill(fake, fake, fake, 1, 1, 4096, 128, ctypes.byref(ix), fake, None, ws, 10, None) == -3
+    assert L.crisp_dense_prefill(fake, fake, fake, 1, 1, 4100, 128, fake, None, ws, big, None) == -2
+    assert L.crisp_dense_prefill(fake, fake, fake, 2, 4, 4096, 128, fake, None, ws, big, None) == -2
+    p = crisp.Params().c()
+    assert L.crisp_prefill(fake, fake, fake, 1, 1, 4096, 128, ctypes.byref(p), fake, None, None, ws, 10, None) == -3
+    assert L.crisp_prefill(fake, fake, fake, 1, 1, 4096, 128, None, fake, None, None, ws, big, None) == -1
+    assert L.crisp_get_status(None, None) == -1
+    assert L.crisp_selftest_timeout(None, 0, 10, None) == -1
+
+
+def test_overflowing_sizes_are_refused(L):
+    p = crisp.Params().c()
+    # N_b (N_b+1)/2 beyond 2^31 entries per head
+    assert L.crisp_workspace_size(1, 1, 128 * 70000, 128, ctypes.byref(p)) == 0
+
+
+def test_compute_calls_fail_loudly_without_the_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(crisp, "_lib", None)
+    monkeypatch.setattr(crisp, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError):
+        crisp.lib()
