@@ -129,6 +129,8 @@ def run_crisp(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
     w = W.WORKLOADS[args.workload]
+    if args.n:
+        w = w.scaled(args.n)
     q, k, v, meta = W.generate(w, device=dev)
     params = crisp.Params()
     ws = crisp.workspace(w.h_q, w.h_kv, w.n, dev)
@@ -179,7 +181,7 @@ def run_crisp(args):
 
     # end to end through the public API: pinned host inputs -> device, prefill, output -> host
     e2e = None
-    if rank == 0 or world > 1:
+    if args.e2e:
         qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
         oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
         qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
@@ -353,6 +355,8 @@ def main():
     ap.add_argument("--impl", default="crisp", choices=["crisp", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--n", type=int, default=0, help="run the workload's generator at another length")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
