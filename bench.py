@@ -30,8 +30,8 @@ from dynamic_block_sparse_proxy_b200 import workloads as W  # noqa: E402
 
 METRIC = "prefill tokens/s per layer (select+sparse attn) at 128k; % bf16 peak, % HBM BW"
 DEFAULT_WORKLOAD = "llama8b_128k"
-# kernels per step: proxy pass, routing, 8 for the PE cut, 5 for the merge, attention
-KERNELS_PER_STEP = 16
+# kernels per step: proxy pass, 3 for routing, 8 for the PE cut, 5 for the merge, attention
+KERNELS_PER_STEP = 18
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 

@@ -222,4 +222,5 @@ def selftest_timeout(ws: torch.Tensor, limit_ns: int) -> int:
 
 
 __all__ = ["Params", "Index", "CrispError", "lib", "workspace_size", "workspace", "select", "sparse_prefill",
-           "prefill", "dense_prefill", "get_status", "check_status", "selftest_timeout", "EXPORTED", "LIB_PATH"]
+           "prefill", "dense_prefill", "get_status", "check_status", "selftest_timeout",
+           "EXPORTED", "LIB_PATH"]

@@ -100,11 +100,14 @@ int run_select(const void* q, const void* k, const Shape& s, const crisp_params*
   a.chunk_max = at<float>(ws, w.chunk_max);
   a.chunk_tot = at<float>(ws, w.chunk_tot);
   a.row_w = at<float>(ws, w.row_w);
+  a.pv = at<double>(ws, w.pv);
+  a.ps_lo = at<double>(ws, w.ps_lo);
+  a.ps_hi = at<double>(ws, w.ps_hi);
   a.kbar = at<float>(ws, w.kbar);
   a.qbar = at<float>(ws, w.qbar);
   a.pbuf = at<float>(ws, w.pbuf);
   a.hist_cnt = at<uint32_t>(ws, w.hist_cnt);
-  a.hist_mass = at<double>(ws, w.hist_mass);
+  a.hist_mass = at<unsigned long long>(ws, w.hist_mass);
   a.cut = at<CutState>(ws, w.cut);
   a.keep_v = at<uint8_t>(ws, w.keep_v);
   a.keep_s = at<uint8_t>(ws, w.keep_s);

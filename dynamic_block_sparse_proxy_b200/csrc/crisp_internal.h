@@ -16,6 +16,7 @@ constexpr int kB = 128;        // block size (queries and keys)
 constexpr int kD = 128;        // head dimension
 constexpr int kProxyChunk = 16;  // key blocks per proxy CTA
 constexpr int kHistBins = 2048;  // radix-select bins per pass (11, 10, 10 bits)
+constexpr double kMassUnit = 1099511627776.0;  // 2^40: fixed-point scale of histogram masses
 
 struct Shape {
   int h_q, h_kv, n, nb, G, n_chunks;
@@ -35,7 +36,7 @@ struct CutState {
 };
 
 struct Workspace {
-  size_t status, trace, part, chunk_max, chunk_tot, row_w, kbar, qbar, pbuf, hist_cnt, hist_mass, cut,
+  size_t status, trace, part, chunk_max, chunk_tot, row_w, pv, ps_lo, ps_hi, kbar, qbar, pbuf, hist_cnt, hist_mass, cut,
       keep_v, keep_s, cnt, eqcnt, eqbase, idx_route, idx_c, idx_row_ptr, idx_cols, total;
 };
 
@@ -56,6 +57,9 @@ inline Workspace workspace_layout(const Shape& s) {
   w.chunk_max = take(hq * ch * kB * 4);
   w.chunk_tot = take(hq * ch * kB * 4);
   w.row_w = take(hq * ch * kB * 4);
+  w.pv = take(hq * nb * 8);
+  w.ps_lo = take(hq * nb * 8);
+  w.ps_hi = take(hq * nb * 8);
   w.kbar = take((size_t)s.h_kv * nb * kD * 4);
   w.qbar = take(hq * nb * kD * 4);
   w.pbuf = take(hq * (size_t)s.cap * 4);
@@ -86,11 +90,14 @@ struct SelectArgs {
   float* chunk_max;
   float* chunk_tot;
   float* row_w;
+  double* pv;      // vertical block masses
+  double* ps_lo;   // slash block masses from the keys at or below each row's diagonal offset
+  double* ps_hi;   // ... and from the keys above it
   float* kbar;
   float* qbar;
   float* pbuf;
   uint32_t* hist_cnt;
-  double* hist_mass;
+  unsigned long long* hist_mass;  // fixed point, 2^-40 units
   CutState* cut;
   uint8_t* keep_v;
   uint8_t* keep_s;

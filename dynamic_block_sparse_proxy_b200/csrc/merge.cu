@@ -18,8 +18,6 @@
 namespace crisp {
 namespace {
 
-constexpr int T = 128;
-
 struct RowCtx {
   int vs, nb, qb;
   const uint8_t* kv;
@@ -29,14 +27,15 @@ struct RowCtx {
   uint32_t keep_all;
 };
 
+// kv/ks point at the head's keep flags (staged in shared memory); every test is branch-free.
 __device__ __forceinline__ bool vs_sel(const RowCtx& c, int kb) {
-  if (c.nb <= 2 || kb == 0 || kb == c.nb - 1) return true;
-  if (c.kv[kb]) return true;
   const int m0 = c.qb - kb;  // offset block m with qb-m == kb
-  if (m0 == 0 || m0 == c.nb - 1 || c.ks[m0]) return true;
   const int m1 = m0 - 1;     // offset block m with qb-m-1 == kb
-  if (m1 >= 0 && (m1 == 0 || m1 == c.nb - 1 || c.ks[m1])) return true;
-  return false;
+  const bool fixed = c.nb <= 2 || kb == 0 || kb == c.nb - 1 || m0 == 0 || m0 == c.nb - 1 || m1 == 0;
+  const bool v = c.kv[kb] != 0;
+  const bool s0 = c.ks[m0] != 0;
+  const bool s1 = m1 >= 0 && c.ks[m1 >= 0 ? m1 : 0] != 0;
+  return fixed | v | s0 | s1;
 }
 
 // PE: where an entry stands relative to the cut value: 0 below, 1 above, 2 equal. Anchors do not
@@ -72,94 +71,111 @@ __device__ __forceinline__ long long tie_quota(const SelectArgs& a, int h) {
   return (a.route[h] || a.s.nb <= 2 || cs.keep_all) ? 0 : (long long)cs.t_eq;
 }
 
-// Block-wide exclusive scan of a 0/1 flag over 128 threads; returns the prefix, total in *tot.
-__device__ __forceinline__ int scan128(int flag, int* wsum, int* tot) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const unsigned bal = __ballot_sync(0xffffffffu, flag);
-  const int pre = __popc(bal & ((1u << lane) - 1u));
-  __syncthreads();
-  if (lane == 0) wsum[w] = __popc(bal);
-  __syncthreads();
-  int off = 0, t = 0;
-#pragma unroll
-  for (int i = 0; i < T / 32; ++i) {
-    if (i < w) off += wsum[i];
-    t += wsum[i];
+// One warp per row, ROWS rows per CTA. Walks row qb of head h in key-block order, 32 blocks per
+// step, and calls emit(kb, position) for every selected block; returns the row's count. Entries
+// tied with the cut value are ranked over the whole head in (qb, kb) order, starting from
+// eqbase[qb]; the first t_eq of them are kept.
+constexpr int ROWS = 8;
+// The head's keep flags staged in shared memory (all rows of a CTA share one head).
+constexpr int kMaxStagedBlocks = 8192;
+__device__ __forceinline__ void stage_flags(const SelectArgs& a, int h, uint8_t* skv, uint8_t* sks) {
+  const int nb = a.s.nb;
+  if (nb > kMaxStagedBlocks) return;
+  const uint8_t* gv = a.keep_v + (size_t)h * nb;
+  const uint8_t* gs = a.keep_s + (size_t)h * nb;
+  for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+    skv[i] = gv[i];
+    sks[i] = gs[i];
   }
-  *tot = t;
-  return off + pre;
+  __syncthreads();
 }
 
-// Walks row qb of head h in key-block order and calls emit(kb) for every selected block.
-// Entries tied with the cut value are ranked over the whole head in (qb, kb) order, starting
-// from eqbase[qb]; the first t_eq of them are kept.
 template <typename Emit>
-__device__ __forceinline__ int walk_row(const SelectArgs& a, int h, int qb, long long erank, Emit emit) {
-  const RowCtx c = make_ctx(a, h, qb);
+__device__ __forceinline__ int walk_row(const SelectArgs& a, int h, int qb, long long erank, const uint8_t* skv,
+                                        const uint8_t* sks, Emit emit) {
+  RowCtx c = make_ctx(a, h, qb);
+  if (a.s.nb <= kMaxStagedBlocks) {
+    c.kv = skv;
+    c.ks = sks;
+  }
   const bool vsrow = c.vs || a.s.nb <= 2;
   const long long t_eq = tie_quota(a, h);
-  __shared__ int wsum[T / 32];
+  // With at most one entry equal to the cut value it is always kept (t_eq >= 1): no ranking.
+  const bool rank_ties = !vsrow && a.cut[h].count_eq > 1;
+  const int lane = threadIdx.x & 31;
+  const unsigned below = (1u << lane) - 1u;
   int count = 0;
-  for (int base = 0; base <= qb; base += T) {
-    const int kb = base + threadIdx.x;
-    int sel = 0, eqf = 0;
-    if (kb <= qb) {
-      if (vsrow) {
-        sel = vs_sel(c, kb);
-      } else {
-        const int f = pe_cut_flag(c, kb);
-        sel = (f == 1) || pe_anchor(c, kb);
-        eqf = f == 2;
+  for (int base = 0; base <= qb; base += 128) {
+    // four 32-entry sub-chunks; the pooled scores of a PE row are loaded together
+    int flag[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int kb = base + 32 * u + lane;
+      flag[u] = (kb <= qb && !vsrow) ? pe_cut_flag(c, kb) : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int kb = base + 32 * u + lane;
+      bool sel = false, eqf = false;
+      if (kb <= qb) {
+        if (vsrow) {
+          sel = vs_sel(c, kb);
+        } else {
+          sel = flag[u] == 1 || pe_anchor(c, kb) || (flag[u] == 2 && !rank_ties);
+          eqf = rank_ties && flag[u] == 2;
+        }
       }
+      if (rank_ties) {
+        const unsigned eb = __ballot_sync(0xffffffffu, eqf);
+        if (eqf && erank + __popc(eb & below) < t_eq) sel = true;
+        erank += __popc(eb);
+      }
+      const unsigned sb = __ballot_sync(0xffffffffu, sel);
+      if (sel) emit(kb, count + __popc(sb & below));
+      count += __popc(sb);
     }
-    if (!vsrow) {
-      int etot;
-      const int epre = scan128(eqf, wsum, &etot);
-      if (eqf && erank + epre < t_eq) sel = 1;
-      erank += etot;
-    }
-    int stot;
-    const int spre = scan128(sel, wsum, &stot);
-    if (sel) emit(kb, count + spre);
-    count += stot;
   }
   return count;
 }
 
-// Pass 1: entries of each PE row that tie with the cut value.
-__global__ void __launch_bounds__(T) merge_ties_kernel(const SelectArgs a) {
-  const int qb = blockIdx.x, h = blockIdx.y;
+// Pass 1: entries of each PE row that tie with the cut value (only heads with >1 such entry).
+__global__ void __launch_bounds__(ROWS * 32) merge_ties_kernel(const SelectArgs a) {
+  const int qb = blockIdx.x * ROWS + (threadIdx.x >> 5), h = blockIdx.y;
+  if (qb >= a.s.nb) return;
+  if (a.cut[h].count_eq <= 1) {
+    if ((threadIdx.x & 31) == 0) a.eqcnt[(size_t)h * a.s.nb + qb] = 0;
+    return;
+  }
   const RowCtx c = make_ctx(a, h, qb);
   int ne = 0;
   if (!(c.vs || a.s.nb <= 2))
-    for (int kb = threadIdx.x; kb <= qb; kb += T) ne += pe_cut_flag(c, kb) == 2;
-  __shared__ int red[T / 32];
+    for (int kb = threadIdx.x & 31; kb <= qb; kb += 32) ne += pe_cut_flag(c, kb) == 2;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ne += __shfl_xor_sync(0xffffffffu, ne, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ne;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int t = 0;
-    for (int i = 0; i < T / 32; ++i) t += red[i];
-    a.eqcnt[(size_t)h * a.s.nb + qb] = t;
-  }
+  if ((threadIdx.x & 31) == 0) a.eqcnt[(size_t)h * a.s.nb + qb] = ne;
 }
 
 // Pass 2: exact number of selected blocks per row.
-__global__ void __launch_bounds__(T) merge_count_kernel(const SelectArgs a) {
-  const int qb = blockIdx.x, h = blockIdx.y;
+__global__ void __launch_bounds__(ROWS * 32) merge_count_kernel(const SelectArgs a) {
+  const int qb = blockIdx.x * ROWS + (threadIdx.x >> 5), h = blockIdx.y;
+  __shared__ uint8_t skv[kMaxStagedBlocks], sks[kMaxStagedBlocks];
+  stage_flags(a, h, skv, sks);
+  if (qb >= a.s.nb) return;
   const long long erank = a.eqbase[(size_t)h * (a.s.nb + 1) + qb];
-  const int n = walk_row(a, h, qb, erank, [](int, int) {});
-  if (threadIdx.x == 0) a.cnt[(size_t)h * a.s.nb + qb] = n;
+  const int n = walk_row(a, h, qb, erank, skv, sks, [](int, int) {});
+  if ((threadIdx.x & 31) == 0) a.cnt[(size_t)h * a.s.nb + qb] = n;
 }
 
 // Pass 3: compaction into the CSR column array.
-__global__ void __launch_bounds__(T) merge_write_kernel(const SelectArgs a) {
-  const int qb = blockIdx.x, h = blockIdx.y;
+__global__ void __launch_bounds__(ROWS * 32) merge_write_kernel(const SelectArgs a) {
+  const int qb = blockIdx.x * ROWS + (threadIdx.x >> 5), h = blockIdx.y;
   const int nb = a.s.nb;
+  __shared__ uint8_t skv[kMaxStagedBlocks], sks[kMaxStagedBlocks];
+  stage_flags(a, h, skv, sks);
+  if (qb >= nb) return;
   const long long erank = a.eqbase[(size_t)h * (nb + 1) + qb];
   int32_t* out = a.cols + (size_t)h * a.s.cap + a.row_ptr[(size_t)h * (nb + 1) + qb];
-  walk_row(a, h, qb, erank, [out](int kb, int pos) { out[pos] = kb; });
+  walk_row(a, h, qb, erank, skv, sks, [out](int kb, int pos) { out[pos] = kb; });
 }
 
 // One CTA per head: exclusive scan of in[h][0..nb) into out[h][0..nb] (out[nb] = total).
@@ -209,11 +225,12 @@ __global__ void __launch_bounds__(1024) scan_rows_kernel(const int* in, int* out
 
 cudaError_t launch_merge(const SelectArgs& a, cudaStream_t st) {
   const Shape& s = a.s;
-  merge_ties_kernel<<<dim3(s.nb, s.h_q), T, 0, st>>>(a);
+  const dim3 rows((s.nb + ROWS - 1) / ROWS, s.h_q);
+  merge_ties_kernel<<<rows, ROWS * 32, 0, st>>>(a);
   scan_rows_kernel<<<s.h_q, 1024, 0, st>>>(a.eqcnt, a.eqbase, s.nb, nullptr);
-  merge_count_kernel<<<dim3(s.nb, s.h_q), T, 0, st>>>(a);
+  merge_count_kernel<<<rows, ROWS * 32, 0, st>>>(a);
   scan_rows_kernel<<<s.h_q, 1024, 0, st>>>(a.cnt, a.row_ptr, s.nb, a.debug);
-  merge_write_kernel<<<dim3(s.nb, s.h_q), T, 0, st>>>(a);
+  merge_write_kernel<<<rows, ROWS * 32, 0, st>>>(a);
   return cudaGetLastError();
 }
 

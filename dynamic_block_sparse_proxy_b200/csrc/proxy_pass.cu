@@ -2,38 +2,46 @@
 // attention A_hat = softmax(Q_hat K^T / sqrt(d)) over a representative query subset, here the
 // last query block; §4: vertical = column means, slash = diagonal means, pooled into blocks).
 //
-// One CTA handles one q-head and a chunk of kProxyChunk key blocks. TMA streams the key blocks
-// of the head's kv-head through a 2-stage ring; one thread issues S = Q_last K_blk^T (128x128x128,
-// bf16 -> fp32) with tcgen05 into a double-buffered TMEM tile; four softmax warps (one query
-// row per thread) read S back, apply the causal mask on the last key block, and accumulate
-// exp2(x - m) with a running row maximum m into two sums per key block: keys at or below the
-// row's diagonal offset (t <= r) and keys above it (t > r). A key at offset t of block kb seen by
-// proxy row r lies on diagonal offset (N_b-1-kb)*B + (r - t), so the first sum belongs to slash
-// block N_b-1-kb and the second to N_b-2-kb; their total is the block's vertical mass. The
-// normalisation by the row's global max and sum happens in the routing kernel.
-//
-// A seventh warp (only in the CTA of the first q-head of each GQA group) sums each K block's
-// rows into the mean-pooled key K_bar used by the Pooled-Estimation path, so K is read once.
+// One CTA handles two q-heads of one GQA group (two "tiles": their last query blocks) against a
+// chunk of kProxyChunk key blocks of the shared kv-head, so every K block is read once for both.
+//   warp 8      TMA producer: both Q tiles, then the chunk's K blocks through a 3-stage ring;
+//   warp 9      one thread issues S_t = Q_t K_blk^T (128x128x128, bf16 -> fp32) into a
+//               double-buffered TMEM tile per head;
+//   warps 0-7   softmax, one warpgroup per head, one proxy row per thread: read the S row with
+//               one TMEM round trip, mask the last key block (key j visible to row r iff
+//               j <= n-B+r), and accumulate exp2(x - m) against a lazy row reference m (it moves
+//               only when a block's maximum exceeds it by more than 2^8) into two sums per key
+//               block: keys at or below the row's diagonal offset (t <= r) and above it (t > r);
+//   warp 10     sums rows of each K block into the mean-pooled key K_bar of the PE path; the
+//               CTAs of one group share the 16 column chunks between them.
+// A key at offset t of block kb seen by proxy row r lies on diagonal offset (N_b-1-kb)*B + (r-t),
+// so the first sum belongs to slash block N_b-1-kb and the second to N_b-2-kb; their total is
+// the block's vertical mass. The per-row normalisation happens in the routing kernels.
 #include "crisp_internal.h"
 #include "sm100.cuh"
 
 namespace crisp {
 namespace {
 
-constexpr int NS = 2;
-constexpr int THREADS = 224;
+constexpr int NS = 3;
+constexpr int THREADS = 352;
+constexpr int PRODUCER_WARP = 8;
+constexpr int MMA_WARP = 9;
+constexpr int POOL_WARP = 10;
 constexpr uint32_t TILE_BYTES = kB * kD * 2;
 constexpr uint32_t HALF_BYTES = TILE_BYTES / 2;
 constexpr float kScaleLog2 = 0.12751743074380045f;  // log2(e) / sqrt(128)
+constexpr float kLazy = 8.0f;
 
 struct __align__(1024) ProxySmem {
-  __nv_bfloat16 q[kB * kD];       // two 128-byte-swizzled halves [128 rows][64 cols]
+  __nv_bfloat16 q[2][kB * kD];  // two 128-byte-swizzled halves [128 rows][64 cols] per tile
   __nv_bfloat16 k[NS][kB * kD];
+  float2 part[2][kProxyChunk][kB];  // per tile, block and row: (lower, upper) sums
   uint64_t q_full;
   uint64_t k_full[NS];
   uint64_t k_empty[NS];
-  uint64_t s_full[2];
-  uint64_t s_free[2];
+  uint64_t s_full[2][2];
+  uint64_t s_free[2][2];
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
@@ -44,7 +52,7 @@ __device__ __forceinline__ void fail(ProxySmem& sm, int* status) {
   *reinterpret_cast<volatile int*>(&sm.abort) = 1;
 }
 
-__global__ void __launch_bounds__(THREADS, 2)
+__global__ void __launch_bounds__(THREADS, 1)
     proxy_pass_kernel(const __grid_constant__ CUtensorMap q_map,
                       const __grid_constant__ CUtensorMap k_map, const SelectArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -53,12 +61,16 @@ __global__ void __launch_bounds__(THREADS, 2)
   const volatile int* abort = &sm.abort;
 
   const Shape& s = a.s;
-  const int h = blockIdx.x % s.h_q;
-  const int chunk = blockIdx.x / s.h_q;
-  const int kv = h / s.G;
+  const int pairs_per_group = (s.G + 1) / 2;
+  const int n_pairs = s.h_kv * pairs_per_group;
+  const int pair = blockIdx.x % n_pairs;
+  const int chunk = blockIdx.x / n_pairs;
+  const int kv = pair / pairs_per_group;
+  const int pig = pair % pairs_per_group;  // pair index within its group
+  const int h0 = kv * s.G + 2 * pig;
+  const int ntiles = (2 * pig + 1 < s.G) ? 2 : 1;
   const int kb0 = chunk * kProxyChunk;
   const int nblk = min(kProxyChunk, s.nb - kb0);
-  const bool pool = (h % s.G) == 0;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
@@ -66,19 +78,20 @@ __global__ void __launch_bounds__(THREADS, 2)
     mbar_init(&sm.q_full, 1);
     for (int i = 0; i < NS; ++i) {
       mbar_init(&sm.k_full[i], 1);
-      mbar_init(&sm.k_empty[i], pool ? 2 : 1);
+      mbar_init(&sm.k_empty[i], 2);  // MMA commit + pooling warp
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.s_free[i], 4);
-    }
+    for (int t = 0; t < 2; ++t)
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&sm.s_full[t][b], 1);
+        mbar_init(&sm.s_free[t][b], 4);
+      }
     mbar_init(&sm.mma_done, 1);
     sm.abort = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == MMA_WARP) {
     __syncwarp();
-    tmem_alloc(&sm.tmem_base, 256);
+    tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -86,15 +99,17 @@ __global__ void __launch_bounds__(THREADS, 2)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  if (warp == 0) {
+  if (warp == PRODUCER_WARP) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&q_map);
       tma_prefetch_desc(&k_map);
-      const int qrow = h * s.n + s.n - kB;
-      mbar_arrive_expect_tx(&sm.q_full, TILE_BYTES);
-      tma_load_2d(&q_map, &sm.q_full, sm.q, 0, qrow);
-      tma_load_2d(&q_map, &sm.q_full, sm.q + kB * 64, 64, qrow);
+      mbar_arrive_expect_tx(&sm.q_full, TILE_BYTES * ntiles);
+      for (int t = 0; t < ntiles; ++t) {
+        const int qrow = (h0 + t) * s.n + s.n - kB;
+        tma_load_2d(&q_map, &sm.q_full, sm.q[t], 0, qrow);
+        tma_load_2d(&q_map, &sm.q_full, sm.q[t] + kB * 64, 64, qrow);
+      }
       int issued = 0;
       for (int j = 0; j < nblk; ++j) {
         const int st = j % NS;
@@ -113,7 +128,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       for (int j = max(0, issued - NS); j < issued; ++j) mbar_wait(&sm.k_full[j % NS], (j / NS) & 1, nullptr);
     }
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp == MMA_WARP) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
@@ -121,20 +136,27 @@ __global__ void __launch_bounds__(THREADS, 2)
       if (!ok) fail(sm, a.status);
       for (int j = 0; ok && j < nblk; ++j) {
         const int st = j % NS, b = j & 1;
-        if (!mbar_wait(&sm.k_full[st], (j / NS) & 1, abort) ||
-            !mbar_wait(&sm.s_free[b], ((j >> 1) & 1) ^ 1, abort)) {
+        if (!mbar_wait(&sm.k_full[st], (j / NS) & 1, abort)) {
           fail(sm, a.status);
           break;
         }
-        tc_fence_after();
-        const uint32_t qa = smem_u32(sm.q), ka = smem_u32(sm.k[st]);
+        for (int t = 0; t < ntiles && ok; ++t) {
+          if (!mbar_wait(&sm.s_free[t][b], ((j >> 1) & 1) ^ 1, abort)) {
+            fail(sm, a.status);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t qa = smem_u32(sm.q[t]), ka = smem_u32(sm.k[st]);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-          umma_ss(tmem + b * 128, desc_kmajor_sw128(qa + off), desc_kmajor_sw128(ka + off), idesc,
-                  kk > 0);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+            umma_ss(tmem + t * 256 + b * 128, desc_kmajor_sw128(qa + off), desc_kmajor_sw128(ka + off), idesc,
+                    kk > 0);
+          }
+          umma_commit(&sm.s_full[t][b]);
         }
-        umma_commit(&sm.s_full[b]);
+        if (!ok) break;
         umma_commit(&sm.k_empty[st]);
       }
       // Never release TMEM under a running MMA: wait (bounded) for all issued work.
@@ -142,112 +164,142 @@ __global__ void __launch_bounds__(THREADS, 2)
       mbar_wait(&sm.mma_done, 0, nullptr);
     }
     __syncwarp();
-  } else if (warp < 6) {
+  } else if (warp < 4 * ntiles) {
     // ------------------------------------------------------------------ softmax rows
+    const int t = warp >> 2;
     const int grp = warp & 3;
     const int r = grp * 32 + lane;
     const uint32_t lane_off = (uint32_t)(grp * 32) << 16;
     float m = -INFINITY;
-    float plo[kProxyChunk], phi[kProxyChunk];
-#pragma unroll
-    for (int jj = 0; jj < kProxyChunk; ++jj) plo[jj] = phi[jj] = 0.f;
     bool ok = true;
     for (int j = 0; j < nblk; ++j) {
       const int b = j & 1;
-      if (!warp_wait(&sm.s_full[b], (j >> 1) & 1, abort)) {
+      if (!warp_wait(&sm.s_full[t][b], (j >> 1) & 1, abort)) {
         fail(sm, a.status);
         ok = false;
         break;
       }
       tc_fence_after();
-      const bool last = (kb0 + j) == s.nb - 1;
+      uint32_t v[4][32];
+      const uint32_t sbase = tmem + t * 256 + b * 128 + lane_off;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(sbase + c * 32, v[c]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.s_free[t][b]);
+
+      if (kb0 + j == s.nb - 1) {
+        // last key block: row r (position n-B+r) sees keys t <= r only
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int q = 0; q < 32; ++q)
+            if (c * 32 + q > r) v[c][q] = __float_as_uint(-INFINITY);
+      }
+      float mx8[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) mx8[q] = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int q = 0; q < 32; ++q) mx8[q & 7] = fmaxf(mx8[q & 7], __uint_as_float(v[c][q]));
+      const float xm = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * kScaleLog2;
+      if (xm > m + kLazy) {
+        // rare: move the reference and rescale this row's earlier blocks
+        const float f = fast_exp2(m - xm);  // 0 while m = -inf
+        for (int jj = 0; jj < j; ++jj) {
+          float2 pv = sm.part[t][jj][r];
+          pv.x *= f;
+          pv.y *= f;
+          sm.part[t][jj][r] = pv;
+        }
+        m = xm;
+      }
+      const float nm = -m;
+      // chunks below the warp's group hold keys t <= r, chunks above hold t > r; chunk grp
+      // straddles the diagonal offset lane by lane
       float lo = 0.f, hi = 0.f;
 #pragma unroll
-      for (int sl = 0; sl < 4; ++sl) {
-        uint32_t v[32];
-        __syncwarp();
-        tmem_ld32(tmem + lane_off + b * 128 + sl * 32, v);
-        tmem_ld_wait();
-        if (sl == 3) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.s_free[b]);
-        }
-        float x[32];
-        float xm = -INFINITY;
+      for (int c = 0; c < 4; ++c) {
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          x[t] = __uint_as_float(v[t]);
-          if (last && (sl * 32 + t) > r) x[t] = -INFINITY;
-          xm = fmaxf(xm, x[t]);
+        for (int q = 0; q < 32; ++q) {
+          const float e = fast_exp2(fmaf(__uint_as_float(v[c][q]), kScaleLog2, nm));
+          v[c][q] = __float_as_uint(e);
+          s4[q & 3] += e;
         }
-        xm *= kScaleLog2;
-        if (xm > m) {
-          const float f = fast_exp2(m - xm);
+        const float sc = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+        if (c < grp) {
+          lo += sc;
+        } else if (c > grp) {
+          hi += sc;
+        } else {
+          float l2[2] = {0.f, 0.f}, h2[2] = {0.f, 0.f};
 #pragma unroll
-          for (int jj = 0; jj < kProxyChunk; ++jj) {
-            plo[jj] *= f;
-            phi[jj] *= f;
+          for (int q = 0; q < 32; ++q) {
+            const float e = __uint_as_float(v[c][q]);
+            if (q <= lane) l2[q & 1] += e; else h2[q & 1] += e;
           }
-          lo *= f;
-          hi *= f;
-          m = xm;
-        }
-#pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          const float e = fast_exp2(fmaf(x[t], kScaleLog2, -m));
-          if (sl * 32 + t <= r) lo += e; else hi += e;
+          lo += l2[0] + l2[1];
+          hi += h2[0] + h2[1];
         }
       }
-#pragma unroll
-      for (int jj = 0; jj < kProxyChunk; ++jj)
-        if (jj == j) {
-          plo[jj] = lo;
-          phi[jj] = hi;
-        }
+      sm.part[t][j][r] = make_float2(lo, hi);
     }
     if (ok) {
+      const int h = h0 + t;
       float tot = 0.f;
-#pragma unroll
-      for (int jj = 0; jj < kProxyChunk; ++jj) {
-        if (jj < nblk) {
-          a.part[((size_t)h * s.nb + kb0 + jj) * kB + r] = make_float2(plo[jj], phi[jj]);
-          tot += plo[jj] + phi[jj];
-        }
+      for (int jj = 0; jj < nblk; ++jj) {
+        const float2 pv = sm.part[t][jj][r];
+        a.part[((size_t)h * s.nb + kb0 + jj) * kB + r] = pv;
+        tot += pv.x + pv.y;
       }
       const size_t ci = ((size_t)h * s.n_chunks + chunk) * kB + r;
       a.chunk_max[ci] = m;
       a.chunk_tot[ci] = tot;
     }
-  } else if (pool) {
+    __syncwarp();
+  } else if (warp == POOL_WARP) {
     // ------------------------------------------------------------------ K block mean (PE path)
-    const int c16 = lane & 15, half = c16 >> 3, ch = c16 & 7, rp = lane >> 4;
+    // Column chunk cc (8 bf16 of each row) belongs to the group's CTA cc % pairs_per_group.
+    // Lane (slot, row group) sums every groups-th row of its chunk; shuffles combine the groups.
+    const int ncc = (16 - pig + pairs_per_group - 1) / pairs_per_group;
+    int groups = 1;
+    while (groups * 2 * ncc <= 32) groups *= 2;
+    const int slot = lane / groups;
+    const int rg = lane % groups;
+    const bool active = slot < ncc;
+    const int cc = pig + slot * pairs_per_group;
+    const int half = cc >> 3, ch = cc & 7;
     for (int j = 0; j < nblk; ++j) {
       const int st = j % NS;
       if (!warp_wait(&sm.k_full[st], (j / NS) & 1, abort)) {
         fail(sm, a.status);
         break;
       }
-      const uint8_t* base = reinterpret_cast<const uint8_t*>(sm.k[st]) + half * HALF_BYTES;
       float acc[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-#pragma unroll 4
-      for (int rr = 0; rr < 64; ++rr) {
-        const int row = 2 * rr + rp;
-        const uint4 u = *reinterpret_cast<const uint4*>(base + sw128_offset(row, ch));
-        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+      if (active) {
+        const uint8_t* base = reinterpret_cast<const uint8_t*>(sm.k[st]) + half * HALF_BYTES;
+        for (int row = rg; row < kB; row += groups) {
+          const uint4 u = *reinterpret_cast<const uint4*>(base + sw128_offset(row, ch));
+          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 f = __bfloat1622float2(p2[i]);
-          acc[2 * i] += f.x;
-          acc[2 * i + 1] += f.y;
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(p2[i]);
+            acc[2 * i] += f.x;
+            acc[2 * i + 1] += f.y;
+          }
         }
       }
+      for (int o = 1; o < groups; o <<= 1)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 16);
-      if (lane < 16) {
-        float4* dst = reinterpret_cast<float4*>(a.kbar + ((size_t)kv * s.nb + kb0 + j) * kD + c16 * 8);
+        for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+      if (active && rg == 0) {
+        float4* dst = reinterpret_cast<float4*>(a.kbar + ((size_t)kv * s.nb + kb0 + j) * kD + cc * 8);
         const float inv = 1.f / kB;
         dst[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
         dst[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
@@ -255,15 +307,15 @@ __global__ void __launch_bounds__(THREADS, 2)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.k_empty[st]);
     }
+    __syncwarp();
   }
 
-  __syncwarp();
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == MMA_WARP) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -275,7 +327,8 @@ cudaError_t launch_proxy_pass(const CUtensorMap& q_map, const CUtensorMap& k_map
   cudaError_t e = cudaFuncSetAttribute(proxy_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.s.h_q * a.s.n_chunks);
+  const int n_pairs = a.s.h_kv * ((a.s.G + 1) / 2);
+  dim3 grid(n_pairs * a.s.n_chunks);
   proxy_pass_kernel<<<grid, THREADS, smem, st>>>(q_map, k_map, a);
   return cudaGetLastError();
 }

@@ -1,7 +1,8 @@
 // route_threshold.cu — per-head routing and the Vertical-Slash noise-floor rule.
 //
 // Inputs are the proxy pass's per-(row, key block) split sums, each relative to its chunk's
-// running row maximum. One CTA per q-head:
+// reference row maximum. Three kernels (row statistics, block masses over many CTAs, and one
+// CTA per q-head for the decisions):
 //   1. per proxy row r: global max M_r and normaliser Z_r over all chunks, and the weight
 //      w = exp2(m_chunk - M_r) / (Z_r * B) that turns a chunk's sums into column-mean mass;
 //   2. p_v[kb] = sum_r w*(lo+hi) (vertical block mass), and the slash block masses
@@ -64,67 +65,74 @@ __device__ int block_argmax(double v, int idx, double* redv, int* redi) {
   return bi;
 }
 
+// 1. Per proxy row r of head h: global reference max M_r over the chunks, normaliser Z_r, and
+//    the weight w = exp2(m_chunk - M_r) / (Z_r * B) that turns a chunk's sums into column-mean mass.
+__global__ void __launch_bounds__(kB) row_stats_kernel(const SelectArgs a) {
+  const Shape& s = a.s;
+  const int h = blockIdx.x, r = threadIdx.x;
+  const float* mc = a.chunk_max + (size_t)h * s.n_chunks * kB;
+  const float* tc = a.chunk_tot + (size_t)h * s.n_chunks * kB;
+  float M = -INFINITY;
+  for (int c = 0; c < s.n_chunks; ++c) M = fmaxf(M, mc[c * kB + r]);
+  double Z = 0.0;
+  for (int c = 0; c < s.n_chunks; ++c) Z += (double)exp2f(mc[c * kB + r] - M) * (double)tc[c * kB + r];
+  float* w = a.row_w + (size_t)h * s.n_chunks * kB;
+  const double inv = 1.0 / (Z * kB);
+  for (int c = 0; c < s.n_chunks; ++c) w[c * kB + r] = (float)((double)exp2f(mc[c * kB + r] - M) * inv);
+}
+
+// 2. Block masses, one warp per key block: p_v[kb] = sum_r w*(lo+hi); the lower-offset halves
+//    belong to slash block N_b-1-kb and the upper ones to N_b-2-kb (CRISP §4, both directions).
+constexpr int MASS_WARPS = 16;
+__global__ void __launch_bounds__(MASS_WARPS * 32) block_mass_kernel(const SelectArgs a) {
+  const Shape& s = a.s;
+  const int h = blockIdx.y, nb = s.nb;
+  const int kb = blockIdx.x * MASS_WARPS + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (kb >= nb) return;
+  const float2* p = a.part + ((size_t)h * nb + kb) * kB;
+  const float* wc = a.row_w + ((size_t)h * s.n_chunks + kb / kProxyChunk) * kB;
+  double lo = 0.0, hi = 0.0;
+#pragma unroll
+  for (int i = 0; i < kB / 32; ++i) {
+    const int r = lane + 32 * i;
+    const float2 v = p[r];
+    const double ww = wc[r];
+    lo += (double)v.x * ww;
+    hi += (double)v.y * ww;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo += __shfl_xor_sync(0xffffffffu, lo, o);
+    hi += __shfl_xor_sync(0xffffffffu, hi, o);
+  }
+  if (lane == 0) {
+    a.pv[(size_t)h * nb + kb] = lo + hi;
+    a.ps_lo[(size_t)h * nb + nb - 1 - kb] = lo;
+    a.ps_hi[(size_t)h * nb + (nb - 2 - kb >= 0 ? nb - 2 - kb : nb - 1)] = nb - 2 - kb >= 0 ? hi : 0.0;
+  }
+}
+
+// 3. Per head: C_struct, route, noise floors, keep flags (+ top-up).
 __global__ void __launch_bounds__(THREADS) route_threshold_kernel(const SelectArgs a) {
   extern __shared__ double dsm[];
   const Shape& s = a.s;
   const int nb = s.nb, h = blockIdx.x, tid = threadIdx.x;
-  double* pv = dsm;             // [nb]
-  double* ps = dsm + nb;        // [nb]  lower-offset halves, then totals
-  double* ps_hi = dsm + 2 * nb; // [nb]
+  double* pv = dsm;       // [nb]
+  double* ps = dsm + nb;  // [nb]
   __shared__ double red[NWARP];
   __shared__ double redv[NWARP];
   __shared__ int redi[NWARP];
-
-  // 1. row statistics and per-chunk weights
-  if (tid < kB) {
-    const float* mc = a.chunk_max + (size_t)h * s.n_chunks * kB;
-    const float* tc = a.chunk_tot + (size_t)h * s.n_chunks * kB;
-    float M = -INFINITY;
-    for (int c = 0; c < s.n_chunks; ++c) M = fmaxf(M, mc[c * kB + tid]);
-    double Z = 0.0;
-    for (int c = 0; c < s.n_chunks; ++c) Z += (double)exp2f(mc[c * kB + tid] - M) * (double)tc[c * kB + tid];
-    float* w = a.row_w + (size_t)h * s.n_chunks * kB;
-    const double inv = 1.0 / (Z * kB);
-    for (int c = 0; c < s.n_chunks; ++c) w[c * kB + tid] = (float)((double)exp2f(mc[c * kB + tid] - M) * inv);
-  }
-  for (int i = tid; i < nb; i += THREADS) ps_hi[i] = 0.0;
-  __syncthreads();
-
-  // 2. block masses
-  const int warp = tid >> 5, lane = tid & 31;
-  const float* w = a.row_w + (size_t)h * s.n_chunks * kB;
-  for (int kb = warp; kb < nb; kb += NWARP) {
-    const float2* p = a.part + ((size_t)h * nb + kb) * kB;
-    const float* wc = w + (size_t)(kb / kProxyChunk) * kB;
-    double lo = 0.0, hi = 0.0;
-#pragma unroll
-    for (int i = 0; i < kB / 32; ++i) {
-      const int r = lane + 32 * i;
-      const float2 v = p[r];
-      const double ww = wc[r];
-      lo += (double)v.x * ww;
-      hi += (double)v.y * ww;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      lo += __shfl_xor_sync(0xffffffffu, lo, o);
-      hi += __shfl_xor_sync(0xffffffffu, hi, o);
-    }
-    if (lane == 0) {
-      pv[kb] = lo + hi;
-      ps[nb - 1 - kb] = lo;
-      if (nb - 2 - kb >= 0) ps_hi[nb - 2 - kb] = hi;
-    }
+  for (int i = tid; i < nb; i += THREADS) {
+    pv[i] = a.pv[(size_t)h * nb + i];
+    ps[i] = a.ps_lo[(size_t)h * nb + i] + (i == nb - 1 ? 0.0 : a.ps_hi[(size_t)h * nb + i]);
   }
   __syncthreads();
-  for (int i = tid; i < nb; i += THREADS) ps[i] += ps_hi[i];
-  __syncthreads();
 
-  // 3. C_struct and route
+  // C_struct and route
   const double C = nb >= 2 ? pv[0] + pv[nb - 1] : pv[0];
   const int vs = C >= (double)a.tau ? 1 : 0;
 
-  // 4. noise floors
+  // noise floors
   double mu_v = 0.0, mu_s = 0.0;
   if (nb >= 3) {
     double rv = 0.0, rs = 0.0;
@@ -138,7 +146,7 @@ __global__ void __launch_bounds__(THREADS) route_threshold_kernel(const SelectAr
     mu_s = rs / (nb - 2);
   }
 
-  // 5. keep flags (+ top-up)
+  // keep flags (+ top-up)
   uint8_t* kv_out = a.keep_v + (size_t)h * nb;
   uint8_t* ks_out = a.keep_s + (size_t)h * nb;
   const double alpha = (double)a.alpha;
@@ -200,7 +208,9 @@ __global__ void __launch_bounds__(THREADS) route_threshold_kernel(const SelectAr
 }  // namespace
 
 cudaError_t launch_route_threshold(const SelectArgs& a, cudaStream_t st) {
-  const size_t smem = (size_t)3 * a.s.nb * sizeof(double);
+  row_stats_kernel<<<a.s.h_q, kB, 0, st>>>(a);
+  block_mass_kernel<<<dim3((a.s.nb + MASS_WARPS - 1) / MASS_WARPS, a.s.h_q), MASS_WARPS * 32, 0, st>>>(a);
+  const size_t smem = (size_t)2 * a.s.nb * sizeof(double);
   cudaError_t e = cudaFuncSetAttribute(route_threshold_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
