@@ -22,7 +22,8 @@ STATUS_NAMES = {
     -4: "CRISP_ERR_CUDA", -5: "CRISP_ERR_DEVICE_TIMEOUT", -6: "CRISP_ERR_OVERFLOW", -7: "CRISP_ERR_DEVICE_CHECK",
 }
 EXPORTED = ["crisp_workspace_size", "crisp_select", "crisp_sparse_prefill", "crisp_prefill",
-            "crisp_dense_prefill", "crisp_get_status", "crisp_status_string", "crisp_selftest_timeout"]
+            "crisp_dense_prefill", "crisp_get_status", "crisp_status_string", "crisp_selftest_timeout",
+            "crisp_select_noalloc"]
 
 
 class CrispError(RuntimeError):

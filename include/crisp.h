@@ -141,6 +141,27 @@ const char* crisp_status_string(int status);
  */
 int crisp_selftest_timeout(void* ws, size_t ws_bytes, uint64_t limit_ns, void* stream);
 
+/*
+ * Index selection that allocates nothing, for callers that must not call cudaMalloc: code running
+ * under a memory manager that owns every device byte (a serving engine's pre-reserved pool), or a
+ * latency-critical path that cannot afford the device synchronisation an allocation implies. The
+ * paper has no counterpart; this is a deployment variant of crisp_select.
+ *   - Same inputs and outputs as crisp_select; instead of a workspace it uses one scratch array of
+ *     32 MiB inside the library (a file-scope device array: every GPU that loads the library holds
+ *     it until the process exits). Shapes whose workspace (crisp_workspace_size) exceeds 32 MiB
+ *     return CRISP_ERR_WORKSPACE without launching anything.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ *     that device current; make that first call before any stream capture.
+ *   - All calls share the array and it keeps the last call's contents; the call clears what must
+ *     start at zero. Calls that overlap on the GPU (other streams, other threads) race on it.
+ *   - device_status: NULL, or a device int the caller has zeroed; a device-side failure stores its
+ *     negative status code there (first failure wins). With NULL such failures go unreported.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ */
+int crisp_select_noalloc(const void* q, const void* k, int h_q, int h_kv, int n, int d,
+                         const crisp_params* params, const crisp_index* out, int* device_status,
+                         void* stream);
+
 #ifdef __cplusplus
 }
 #endif
