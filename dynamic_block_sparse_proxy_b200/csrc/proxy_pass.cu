@@ -9,10 +9,11 @@
 //               double-buffered TMEM tile per head;
 //   warps 0-7   softmax, one warpgroup per head, one proxy row per thread: read the S row with
 //               one TMEM round trip, mask the last key block (key j visible to row r iff
-//               j <= n-B+r), and accumulate exp2(x - m) against a lazy row reference m (it moves
-//               only when a block's maximum exceeds it by more than 2^8) into two sums per key
-//               block: keys at or below the row's diagonal offset (t <= r) and above it (t > r);
-//   warp 10     sums rows of each K block into the mean-pooled key K_bar of the PE path; the
+//               j <= n-B+r), and accumulate exp2(x - m) against a lagging row reference m (set
+//               by the chunk's first block, moved only when a block's sum would leave
+//               [0, 2^64]) into two sums per key block: keys at or below the row's diagonal
+//               offset (t <= r) and above it (t > r);
+//   warps 10-11 sum rows of each K block into the mean-pooled key K_bar of the PE path; the
 //               CTAs of one group share the 16 column chunks between them.
 // A key at offset t of block kb seen by proxy row r lies on diagonal offset (N_b-1-kb)*B + (r-t),
 // so the first sum belongs to slash block N_b-1-kb and the second to N_b-2-kb; their total is
@@ -24,14 +25,13 @@ namespace crisp {
 namespace {
 
 constexpr int NS = 3;
-constexpr int THREADS = 352;
+constexpr int THREADS = 384;
 constexpr int PRODUCER_WARP = 8;
 constexpr int MMA_WARP = 9;
-constexpr int POOL_WARP = 10;
+constexpr int POOL_WARP = 10;   // and 11: two warps share the pooling
 constexpr uint32_t TILE_BYTES = kB * kD * 2;
 constexpr uint32_t HALF_BYTES = TILE_BYTES / 2;
 constexpr float kScaleLog2 = 0.12751743074380045f;  // log2(e) / sqrt(128)
-constexpr float kLazy = 8.0f;
 
 struct __align__(1024) ProxySmem {
   __nv_bfloat16 q[2][kB * kD];  // two 128-byte-swizzled halves [128 rows][64 cols] per tile
@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(&sm.q_full, 1);
     for (int i = 0; i < NS; ++i) {
       mbar_init(&sm.k_full[i], 1);
-      mbar_init(&sm.k_empty[i], 2);  // MMA commit + pooling warp
+      mbar_init(&sm.k_empty[i], 3);  // MMA commit + two pooling warps
     }
     for (int t = 0; t < 2; ++t)
       for (int b = 0; b < 2; ++b) {
@@ -180,72 +180,85 @@ __global__ void __launch_bounds__(THREADS, 1)
         break;
       }
       tc_fence_after();
+      // Exponentials use the row reference m of the chunk's earlier blocks without this block's
+      // maximum (fp32 keeps them exact until they overflow); the first block sets m from its
+      // maximum, and a block whose sum would leave [0, 2^64] is redone against its maximum with
+      // the earlier partial sums rescaled. S stays in TMEM until the block is done.
       uint32_t v[4][32];
       const uint32_t sbase = tmem + t * 256 + b * 128 + lane_off;
+      const bool last = kb0 + j == s.nb - 1;
+      bool need_max = (m == -INFINITY);
+      float lo = 0.f, hi = 0.f;
+      for (int attempt = 0; attempt < 2; ++attempt) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(sbase + c * 32, v[c]);
-      tmem_ld_wait();
+        for (int c = 0; c < 4; ++c) tmem_ld32(sbase + c * 32, v[c]);
+        tmem_ld_wait();
+        if (last) {
+          // last key block: row r (position n-B+r) sees keys t <= r only
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+              if (c * 32 + q > r) v[c][q] = __float_as_uint(-INFINITY);
+        }
+        if (need_max) {
+          float mx8[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) mx8[q] = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int q = 0; q < 32; ++q) mx8[q & 7] = fmaxf(mx8[q & 7], __uint_as_float(v[c][q]));
+          const float xm = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * kScaleLog2;
+          if (xm > m) {
+            const float f = fast_exp2(m - xm);  // 0 while m = -inf
+            for (int jj = 0; jj < j; ++jj) {
+              float2 pv = sm.part[t][jj][r];
+              pv.x *= f;
+              pv.y *= f;
+              sm.part[t][jj][r] = pv;
+            }
+            m = xm;
+          }
+        }
+        const float nm = -m;
+        // chunks below the warp's group hold keys t <= r, chunks above hold t > r; chunk grp
+        // straddles the diagonal offset lane by lane
+        lo = 0.f;
+        hi = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            const float e = fast_exp2(fmaf(__uint_as_float(v[c][q]), kScaleLog2, nm));
+            v[c][q] = __float_as_uint(e);
+            s4[q & 3] += e;
+          }
+          const float sc = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+          if (c < grp) {
+            lo += sc;
+          } else if (c > grp) {
+            hi += sc;
+          } else {
+            float l2[2] = {0.f, 0.f}, h2[2] = {0.f, 0.f};
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+              const float e = __uint_as_float(v[c][q]);
+              if (q <= lane) l2[q & 1] += e; else h2[q & 1] += e;
+            }
+            lo += l2[0] + l2[1];
+            hi += h2[0] + h2[1];
+          }
+        }
+        const bool redo = !need_max && !(lo + hi <= 18446744073709551616.0f);  // 2^64, or inf / nan
+        if (!__any_sync(0xffffffffu, redo)) break;
+        need_max = true;
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.s_free[t][b]);
-
-      if (kb0 + j == s.nb - 1) {
-        // last key block: row r (position n-B+r) sees keys t <= r only
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int q = 0; q < 32; ++q)
-            if (c * 32 + q > r) v[c][q] = __float_as_uint(-INFINITY);
-      }
-      float mx8[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) mx8[q] = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int q = 0; q < 32; ++q) mx8[q & 7] = fmaxf(mx8[q & 7], __uint_as_float(v[c][q]));
-      const float xm = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * kScaleLog2;
-      if (xm > m + kLazy) {
-        // rare: move the reference and rescale this row's earlier blocks
-        const float f = fast_exp2(m - xm);  // 0 while m = -inf
-        for (int jj = 0; jj < j; ++jj) {
-          float2 pv = sm.part[t][jj][r];
-          pv.x *= f;
-          pv.y *= f;
-          sm.part[t][jj][r] = pv;
-        }
-        m = xm;
-      }
-      const float nm = -m;
-      // chunks below the warp's group hold keys t <= r, chunks above hold t > r; chunk grp
-      // straddles the diagonal offset lane by lane
-      float lo = 0.f, hi = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float s4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          const float e = fast_exp2(fmaf(__uint_as_float(v[c][q]), kScaleLog2, nm));
-          v[c][q] = __float_as_uint(e);
-          s4[q & 3] += e;
-        }
-        const float sc = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-        if (c < grp) {
-          lo += sc;
-        } else if (c > grp) {
-          hi += sc;
-        } else {
-          float l2[2] = {0.f, 0.f}, h2[2] = {0.f, 0.f};
-#pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            const float e = __uint_as_float(v[c][q]);
-            if (q <= lane) l2[q & 1] += e; else h2[q & 1] += e;
-          }
-          lo += l2[0] + l2[1];
-          hi += h2[0] + h2[1];
-        }
-      }
       sm.part[t][j][r] = make_float2(lo, hi);
     }
     if (ok) {
@@ -261,17 +274,20 @@ __global__ void __launch_bounds__(THREADS, 1)
       a.chunk_tot[ci] = tot;
     }
     __syncwarp();
-  } else if (warp == POOL_WARP) {
+  } else if (warp >= POOL_WARP) {
     // ------------------------------------------------------------------ K block mean (PE path)
-    // Column chunk cc (8 bf16 of each row) belongs to the group's CTA cc % pairs_per_group.
-    // Lane (slot, row group) sums every groups-th row of its chunk; shuffles combine the groups.
-    const int ncc = (16 - pig + pairs_per_group - 1) / pairs_per_group;
+    // Column chunk cc (8 bf16 of each row) belongs to the group's CTA cc % pairs_per_group, and
+    // within the CTA to pooling warp (its slot index) % 2. Lane (slot, row group) sums every
+    // groups-th row of its chunk; shuffles combine the row groups.
+    const int pw = warp - POOL_WARP;
+    const int ncc_cta = (16 - pig + pairs_per_group - 1) / pairs_per_group;
+    const int ncc = (ncc_cta - pw + 1) / 2;
     int groups = 1;
-    while (groups * 2 * ncc <= 32) groups *= 2;
+    while (groups < 32 && groups * 2 * ncc <= 32) groups *= 2;
     const int slot = lane / groups;
     const int rg = lane % groups;
     const bool active = slot < ncc;
-    const int cc = pig + slot * pairs_per_group;
+    const int cc = pig + (2 * slot + pw) * pairs_per_group;
     const int half = cc >> 3, ch = cc & 7;
     for (int j = 0; j < nblk; ++j) {
       const int st = j % NS;
@@ -283,15 +299,24 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = 0.f;
       if (active) {
+        // 128/groups rows per lane, eight independent 16-byte loads in flight
         const uint8_t* base = reinterpret_cast<const uint8_t*>(sm.k[st]) + half * HALF_BYTES;
-        for (int row = rg; row < kB; row += groups) {
-          const uint4 u = *reinterpret_cast<const uint4*>(base + sw128_offset(row, ch));
-          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+        for (int row0 = rg; row0 < kB; row0 += 8 * groups) {
+          uint4 u[8];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float2 f = __bfloat1622float2(p2[i]);
-            acc[2 * i] += f.x;
-            acc[2 * i + 1] += f.y;
+          for (int x = 0; x < 8; ++x) {
+            const int row = row0 + x * groups;
+            u[x] = row < kB ? *reinterpret_cast<const uint4*>(base + sw128_offset(row, ch)) : make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int x = 0; x < 8; ++x) {
+            const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&u[x]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 f = __bfloat1622float2(p2[i]);
+              acc[2 * i] += f.x;
+              acc[2 * i + 1] += f.y;
+            }
           }
         }
       }

@@ -8,41 +8,46 @@
 // block is in its own list.
 //   warps 0-3   softmax of tile 0, warps 4-7 softmax of tile 1 (one query row per thread):
 //               read S from TMEM, mask the diagonal block (key j visible to query i iff j <= i),
-//               online softmax in the exp2 domain with a lazy maximum (O and the row sum are
-//               rescaled only when the maximum grows by more than 2^8), write bf16 P back into
-//               the tile's S columns; at the end scale O by 1/l, store bf16 O and the LSE;
-//   warp 8      TMA producer: both Q tiles once, then K and V blocks of the union through a
-//               2-stage ring (128-byte swizzle, two 64-column boxes per 128x128 tile);
-//   warp 9      one thread issues the UMMAs in ping-pong order: for each tile, O_t += P_t V of
-//               the previous step (A operand read from TMEM), then S_t = Q_t K^T of this step,
-//               so the tensor core works on one tile while the other tile's softmax runs.
+//               online softmax in the exp2 domain against a lagging row reference (O and the
+//               row sum are rescaled only when a block's exponentials would leave [0, 2^64]),
+//               write bf16 P back into the tile's S columns; at the end scale O by 1/l, store
+//               bf16 O and the LSE;
+//   warp 8      TMA producer of both Q tiles once, then the K blocks of the union through a
+//               3-stage ring (128-byte swizzle, two 64-column boxes per 128x128 tile);
+//   warp 11     TMA producer of the V blocks through a 2-stage ring;
+//   warps 9-10  one thread per tile issues that tile's UMMAs: O_t += P_t V of the previous step
+//               (A operand read from TMEM), then S_t = Q_t K^T of this step; the two tiles run
+//               out of phase, so the tensor core works on one while the other's softmax runs.
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; P_t is packed bf16 over S_t.
 // tcgen05 MMAs issued by one thread execute in order, so S_t is overwritten only after the PV
 // that read P_t from the same columns, and the commit that signals S_t also covers that PV.
+// Both tiles' MMAs run on the same tensor core, interleaved as their issuers go.
 #include "crisp_internal.h"
 #include "sm100.cuh"
 
 namespace crisp {
 namespace {
 
-constexpr int NS = 2;
-constexpr int THREADS = 320;
-constexpr int PRODUCER_WARP = 8;
-constexpr int MMA_WARP = 9;
+constexpr int NSK = 3;  // K ring depth
+constexpr int NSV = 2;  // V ring depth
+constexpr int THREADS = 384;
+constexpr int PRODUCER_WARP = 8;     // Q and K
+constexpr int V_PRODUCER_WARP = 11;  // V
+constexpr int MMA_WARP = 9;  // and 10: one issuing warp per tile
 constexpr uint32_t TILE_BYTES = kB * kD * 2;
 constexpr uint32_t HALF_BYTES = TILE_BYTES / 2;
-constexpr float kLazyRescale = 8.0f;  // log2 units
 constexpr float kLn2 = 0.6931471805599453f;
 
 struct __align__(1024) AttnSmem {
   __nv_bfloat16 q[2][kB * kD];
-  __nv_bfloat16 k[NS][kB * kD];
-  __nv_bfloat16 v[NS][kB * kD];
+  __nv_bfloat16 k[NSK][kB * kD];
+  __nv_bfloat16 v[NSV][kB * kD];
   uint64_t q_full;
-  uint64_t k_full[NS], k_empty[NS];
-  uint64_t v_full[NS], v_empty[NS];
+  uint64_t k_full[NSK], k_empty[NSK];
+  uint64_t v_full[NSV], v_empty[NSV];
   uint64_t s_full[2], p_full[2];
-  uint64_t o_done;
+  uint64_t o_done[2];
+  uint64_t turn[2][4];  // softmax turn handoff between the tiles, per sub-partition
   uint32_t tmem_base;
   int abort;
 };
@@ -92,14 +97,17 @@ __global__ void __launch_bounds__(THREADS, 1)
   const Shape& s = a.s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // work item: (pair of q-heads of one GQA group, query block), longest rows first
+  // work item: (kv-head, query block, pair of q-heads of its GQA group). kv-heads run one
+  // after another and, within one, the longest rows first: the CTAs resident at a time stream
+  // the same kv-head's K and V, which then stay in L2 instead of all heads competing for it.
   const int pairs_per_group = (s.G + 1) / 2;
-  const int n_pairs = s.h_kv * pairs_per_group;
-  const int pair = blockIdx.x % n_pairs;
-  const int qb = s.nb - 1 - (int)(blockIdx.x / n_pairs);
-  const int kv = pair / pairs_per_group;
-  const int h0 = kv * s.G + 2 * (pair % pairs_per_group);
-  const int ntiles = (2 * (pair % pairs_per_group) + 1 < s.G) ? 2 : 1;
+  const int per_kv = pairs_per_group * s.nb;
+  const int kv = (int)(blockIdx.x / per_kv);
+  const int rem = (int)(blockIdx.x % per_kv);
+  const int qb = s.nb - 1 - rem / pairs_per_group;
+  const int pig = rem % pairs_per_group;
+  const int h0 = kv * s.G + 2 * pig;
+  const int ntiles = (2 * pig + 1 < s.G) ? 2 : 1;
   const bool dense = a.dense != 0;
 
   TileList tl[2];
@@ -124,17 +132,22 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.q_full, 1);
-    for (int i = 0; i < NS; ++i) {
+    for (int i = 0; i < NSK; ++i) {
       mbar_init(&sm.k_full[i], 1);
-      mbar_init(&sm.k_empty[i], 1);
+      mbar_init(&sm.k_empty[i], ntiles);  // one release per tile
+    }
+    for (int i = 0; i < NSV; ++i) {
       mbar_init(&sm.v_full[i], 1);
-      mbar_init(&sm.v_empty[i], 1);
+      mbar_init(&sm.v_empty[i], ntiles);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&sm.s_full[t], 1);
       mbar_init(&sm.p_full[t], 4);
     }
-    mbar_init(&sm.o_done, 1);
+    mbar_init(&sm.o_done[0], 1);
+    mbar_init(&sm.o_done[1], 1);
+    for (int t = 0; t < 2; ++t)
+      for (int g = 0; g < 4; ++g) mbar_init(&sm.turn[t][g], 1);
     sm.abort = 0;
     fence_mbar_init();
   }
@@ -152,11 +165,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     // Malformed row: report it and emit nothing for this block.
     if (threadIdx.x == 0) record_status(a.status, CRISP_ERR_DEVICE_CHECK);
   } else if (warp == PRODUCER_WARP) {
-    // ------------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------------ TMA producer: Q, K
     if (lane == 0) {
       tma_prefetch_desc(&q_map);
       tma_prefetch_desc(&k_map);
-      tma_prefetch_desc(&v_map);
       mbar_arrive_expect_tx(&sm.q_full, TILE_BYTES * ntiles);
       for (int t = 0; t < ntiles; ++t) {
         const int qrow = (h0 + t) * s.n + qb * kB;
@@ -171,10 +183,10 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
       }
       UnionWalk u{{tl[0], tl[1]}, {0, 0}, dense, qb};
-      int kb, mask, nk = 0, nv = 0;
+      int kb, mask, nk = 0;
       for (int step = 0; u.next(kb, mask); ++step) {
-        const int st = step % NS;
-        const uint32_t par = ((step / NS) & 1) ^ 1;
+        const int st = step % NSK;
+        const uint32_t par = ((step / NSK) & 1) ^ 1;
         const int krow = kv * s.n + kb * kB;
         trace_mark(a.trace, 0, 0, 1, step);
         if (!mbar_wait(&sm.k_empty[st], par, abort)) { fail(sm, a.status, CRISP_ERR_DEVICE_TIMEOUT); break; }
@@ -182,92 +194,112 @@ __global__ void __launch_bounds__(THREADS, 1)
         tma_load_2d(&k_map, &sm.k_full[st], sm.k[st], 0, krow);
         tma_load_2d(&k_map, &sm.k_full[st], sm.k[st] + kB * 64, 64, krow);
         nk = step + 1;
-        trace_mark(a.trace, 0, 0, 2, step);
+      }
+      // Never leave with copies in flight (bounded waits on the last use of each slot).
+      trace_mark(a.trace, 0, 0, 4, 0);
+      mbar_wait(&sm.q_full, 0, nullptr);
+      for (int i = max(0, nk - NSK); i < nk; ++i) mbar_wait(&sm.k_full[i % NSK], (i / NSK) & 1, nullptr);
+      trace_mark(a.trace, 0, 0, 5, 0);
+    }
+    __syncwarp();
+  } else if (warp == V_PRODUCER_WARP) {
+    // ------------------------------------------------------------------ TMA producer: V
+    // Its own thread, so a V slot that is released late never holds back the next K load.
+    if (lane == 0) {
+      tma_prefetch_desc(&v_map);
+      UnionWalk u{{tl[0], tl[1]}, {0, 0}, dense, qb};
+      int kb, mask, nv = 0;
+      for (int step = 0; u.next(kb, mask); ++step) {
+        const int st = step % NSV;
+        const uint32_t par = ((step / NSV) & 1) ^ 1;
+        const int krow = kv * s.n + kb * kB;
+        trace_mark(a.trace, 0, 5, 2, step);
         if (!mbar_wait(&sm.v_empty[st], par, abort)) { fail(sm, a.status, CRISP_ERR_DEVICE_TIMEOUT); break; }
         mbar_arrive_expect_tx(&sm.v_full[st], TILE_BYTES);
         tma_load_2d(&v_map, &sm.v_full[st], sm.v[st], 0, krow);
         tma_load_2d(&v_map, &sm.v_full[st], sm.v[st] + kB * 64, 64, krow);
         nv = step + 1;
       }
-      // Never leave with copies in flight (bounded waits on the last use of each slot).
-      trace_mark(a.trace, 0, 0, 4, 0);
-      mbar_wait(&sm.q_full, 0, nullptr);
-      for (int i = max(0, nk - NS); i < nk; ++i) mbar_wait(&sm.k_full[i % NS], (i / NS) & 1, nullptr);
-      for (int i = max(0, nv - NS); i < nv; ++i) mbar_wait(&sm.v_full[i % NS], (i / NS) & 1, nullptr);
-      trace_mark(a.trace, 0, 0, 5, 0);
+      for (int i = max(0, nv - NSV); i < nv; ++i) mbar_wait(&sm.v_full[i % NSV], (i / NSV) & 1, nullptr);
+      trace_mark(a.trace, 0, 5, 5, 0);
     }
     __syncwarp();
-  } else if (warp == MMA_WARP) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (warp >= MMA_WARP && warp - MMA_WARP < ntiles) {
+    // ------------------------------------------------------------------ MMA issuer of tile t
+    // Each tile has its own issuing thread, so a tile's PV and next QK go out as soon as its own
+    // P is ready instead of waiting for the other tile's turn. K and V slots are released by
+    // both issuers: with a commit after the tile's MMAs that read the slot, or with a plain
+    // arrive for a block the tile skips (after the slot's fill completed, so an arrive never
+    // counts towards an earlier use of the slot).
+    const int t = warp - MMA_WARP;
+    const int role = t ? 4 : 1;
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);
+      const uint32_t bit = 1u << t;
+      const uint32_t s_tmem = tmem + t * 128;
+      const uint32_t o_tmem = tmem + 256 + t * 128;
+      const uint32_t qa = smem_u32(sm.q[t]);
       bool ok = mbar_wait(&sm.q_full, 0, abort);
       if (!ok) fail(sm, a.status, CRISP_ERR_DEVICE_TIMEOUT);
       UnionWalk u{{tl[0], tl[1]}, {0, 0}, dense, qb};
-      int pv_n[2] = {0, 0};  // PV_t issued so far
-      int prev_mask = 0, prev_st = 0, kb = 0, mask = 0, step = 0;
+      int pv_n = 0;  // PV of this tile issued so far
+      int prev_mask = 0, kb = 0, mask = 0, step = 0;
       while (ok) {
         const bool more = u.next(kb, mask);
         if (!more) mask = 0;
-        const int st = step % NS;
-        bool v_ready = false, k_ready = false;
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          if (!ok) continue;
-          if (prev_mask & (1 << t)) {
-            // O_t += P_t V of the previous step; P_t sits in the S_t columns
-            trace_mark(a.trace, 0, 1, 3, step);
-            if (!mbar_wait(&sm.p_full[t], pv_n[t] & 1, abort) ||
-                (!v_ready && !mbar_wait(&sm.v_full[prev_st], ((step - 1) / NS) & 1, abort))) {
-              fail(sm, a.status, CRISP_ERR_DEVICE_TIMEOUT);
-              ok = false;
-              continue;
-            }
-            v_ready = true;
+        const int st = step % NSK;
+        const int prev_vs = (step + NSV - 1) % NSV;
+        if (step > 0) {
+          // V of the previous step: O_t += P_t V (P_t sits in the S_t columns), or skip it
+          trace_mark(a.trace, 0, role, 3, step);
+          const bool use = (prev_mask & bit) != 0;
+          if ((use && !mbar_wait(&sm.p_full[t], pv_n & 1, abort)) ||
+              !mbar_wait(&sm.v_full[prev_vs], ((step - 1) / NSV) & 1, abort)) {
+            fail(sm, a.status, CRISP_ERR_DEVICE_TIMEOUT);
+            break;
+          }
+          if (use) {
             tc_fence_after();
-            const uint32_t va = smem_u32(sm.v[prev_st]);
-            const uint32_t p_tmem = tmem + t * 128;
-            const uint32_t o_tmem = tmem + 256 + t * 128;
+            const uint32_t va = smem_u32(sm.v[prev_vs]);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              umma_ts(o_tmem, p_tmem + kk * 8, desc_mnmajor_sw128(va + kk * 2048, HALF_BYTES), idesc_pv,
-                      (pv_n[t] > 0 || kk > 0) ? 1u : 0u);
-            ++pv_n[t];
-          }
-          if (mask & (1 << t)) {
-            // S_t = Q_t K^T of this step
-            trace_mark(a.trace, 0, 1, 1, step);
-            if (!k_ready && !mbar_wait(&sm.k_full[st], (step / NS) & 1, abort)) {
-              fail(sm, a.status, CRISP_ERR_DEVICE_TIMEOUT);
-              ok = false;
-              continue;
-            }
-            k_ready = true;
-            tc_fence_after();
-            const uint32_t qa = smem_u32(sm.q[t]), ka = smem_u32(sm.k[st]);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-              umma_ss(tmem + t * 128, desc_kmajor_sw128(qa + off), desc_kmajor_sw128(ka + off), idesc_qk,
-                      kk > 0);
-            }
-            umma_commit(&sm.s_full[t]);
+              umma_ts(o_tmem, s_tmem + kk * 8, desc_mnmajor_sw128(va + kk * 2048, HALF_BYTES), idesc_pv,
+                      (pv_n > 0 || kk > 0) ? 1u : 0u);
+            ++pv_n;
+            umma_commit(&sm.v_empty[prev_vs]);
+          } else {
+            mbar_arrive(&sm.v_empty[prev_vs]);
           }
         }
-        if (!ok) break;
-        if (prev_mask) umma_commit(&sm.v_empty[prev_st]);
-        if (mask) umma_commit(&sm.k_empty[st]);
         if (!more) break;
+        // K of this step: S_t = Q_t K^T, or skip it
+        trace_mark(a.trace, 0, role, 1, step);
+        if (!mbar_wait(&sm.k_full[st], (step / NSK) & 1, abort)) {
+          fail(sm, a.status, CRISP_ERR_DEVICE_TIMEOUT);
+          break;
+        }
+        if (mask & bit) {
+          tc_fence_after();
+          const uint32_t ka = smem_u32(sm.k[st]);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+            umma_ss(s_tmem, desc_kmajor_sw128(qa + off), desc_kmajor_sw128(ka + off), idesc_qk, kk > 0);
+          }
+          umma_commit(&sm.s_full[t]);
+          umma_commit(&sm.k_empty[st]);
+        } else {
+          mbar_arrive(&sm.k_empty[st]);
+        }
         prev_mask = mask;
-        prev_st = st;
         ++step;
       }
-      trace_mark(a.trace, 0, 1, 6, step);
+      trace_mark(a.trace, 0, role, 6, step);
       // Never release TMEM under a running MMA: the epilogue and teardown wait for this.
-      umma_commit(&sm.o_done);
-      mbar_wait(&sm.o_done, 0, nullptr);
-      trace_mark(a.trace, 0, 1, 7, step);
+      umma_commit(&sm.o_done[t]);
+      mbar_wait(&sm.o_done[t], 0, nullptr);
+      trace_mark(a.trace, 0, role, 7, step);
     }
     __syncwarp();
   } else if (warp < 4 * ntiles) {
@@ -283,10 +315,26 @@ __global__ void __launch_bounds__(THREADS, 1)
     const float sc = a.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    const TileList my = t ? tl[1] : tl[0];
-    const int L = my.len;
-    for (int i = 0; i < L; ++i) {
-      const int kb = my.at(i, dense, qb);
+    // Warp grp of tile 0 and warp grp of tile 1 share a sub-partition and its exp2 unit; they
+    // take turns over the exponentials of each step of the union walk (tile 0 first), so the
+    // two tiles stay half a cycle apart and one tile's MMAs run during the other's softmax.
+    const bool turns = ntiles == 2;
+    uint64_t* my_turn = &sm.turn[t][grp];
+    uint64_t* next_turn = &sm.turn[t ^ 1][grp];
+    UnionWalk u{{tl[0], tl[1]}, {0, 0}, dense, qb};
+    int kb = 0, mask = 0, i = 0;
+    for (int j = 0; u.next(kb, mask); ++j) {
+      const bool mine = (mask >> t) & 1;
+      const uint32_t turn_parity = (uint32_t)(j & 1) ^ (t == 0 ? 1u : 0u);
+      if (!mine) {
+        if (turns && !warp_wait(my_turn, turn_parity, abort)) {
+          fail(sm, a.status, CRISP_ERR_DEVICE_TIMEOUT);
+          ok = false;
+          break;
+        }
+        if (turns && lane == 0) mbar_arrive(next_turn);
+        continue;
+      }
       if (tracer) trace_mark(a.trace, 0, role, 1, i);
       if (!warp_wait(&sm.s_full[t], i & 1, abort)) {
         fail(sm, a.status, CRISP_ERR_DEVICE_TIMEOUT);
@@ -294,78 +342,97 @@ __global__ void __launch_bounds__(THREADS, 1)
         break;
       }
       tc_fence_after();
-      // S row: all four 32-column loads in flight, one wait (a TMEM round trip is expensive
-      // while the tensor core works on the other tile)
+      // Exponentials use the row reference m of the earlier blocks without looking for this
+      // block's maximum: fp32 (and bf16) share fp32's exponent range, so exp2(x*sc - m) stays
+      // exact as long as it does not overflow. The first block sets m from its maximum; a later
+      // block whose exponentials sum beyond 2^64 (or overflow) is redone against its maximum,
+      // with O and l rescaled. The result is the same softmax either way.
       uint32_t v[4][32];
+      bool need_max = (i == 0), turn_ok = true;
+      float rs = 0.f, alpha = 1.f;
+      for (int attempt = 0; attempt < 2; ++attempt) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(s_tmem + c * 32, v[c]);
-      tmem_ld_wait();
-      if (kb == qb) {
+        for (int c = 0; c < 4; ++c) tmem_ld32(s_tmem + c * 32, v[c]);
+        tmem_ld_wait();
+        // the turn is taken once S is in registers
+        if (attempt == 0 && turns && !warp_wait(my_turn, turn_parity, abort)) {
+          turn_ok = false;
+          break;
+        }
+        if (kb == qb) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj)
+              if (c * 32 + jj > r) v[c][jj] = __float_as_uint(-INFINITY);
+        }
+        if (need_max) {
+          float mx8[8];
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) mx8[jj] = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) mx8[jj & 7] = fmaxf(mx8[jj & 7], __uint_as_float(v[c][jj]));
+          const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * sc;
+          const float m_new = fmaxf(m, mx);
+          alpha = fast_exp2(m - m_new);  // 0 on the first block (m = -inf)
+          m = m_new;
+        }
+        const float nm = -m;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (c * 32 + j > r) v[c][j] = __float_as_uint(-INFINITY);
+          for (int jj = 0; jj < 16; ++jj) {
+            const float e0 = fast_exp2(fmaf(__uint_as_float(v[c][2 * jj]), sc, nm));
+            const float e1 = fast_exp2(fmaf(__uint_as_float(v[c][2 * jj + 1]), sc, nm));
+            acc[jj & 3] += e0 + e1;
+            v[c][jj] = pack_bf16(e0, e1);  // pair jj overwrites register jj, already read
+          }
+        rs = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        const bool redo = !need_max && !(rs <= 18446744073709551616.0f);  // 2^64, or inf / nan
+        if (!__any_sync(0xffffffffu, redo)) break;
+        need_max = true;
       }
-      // row maximum over eight independent chains
-      float mx8[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) mx8[j] = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int j = 0; j < 32; ++j) mx8[j & 7] = fmaxf(mx8[j & 7], __uint_as_float(v[c][j]));
-      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      mx *= sc;
-      float m_new = m;
-      bool rescale = false;
-      if (mx > m + kLazyRescale || m == -INFINITY) {
-        m_new = mx;
-        rescale = (m != -INFINITY);
+      if (!turn_ok) {
+        fail(sm, a.status, CRISP_ERR_DEVICE_TIMEOUT);
+        ok = false;
+        break;
       }
-      const float alpha = fast_exp2(m - m_new);  // 0 on the first block (m = -inf), 1 if kept
-      // P = exp2(x*sc - m), packed to bf16 pairs in place (pair j of a chunk overwrites register
-      // j, already read) and stored over the S columns: keys 32c..32c+31 -> columns 16c..16c+15.
-      const float nm = -m_new;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float e0 = fast_exp2(fmaf(__uint_as_float(v[c][2 * j]), sc, nm));
-          const float e1 = fast_exp2(fmaf(__uint_as_float(v[c][2 * j + 1]), sc, nm));
-          acc[j & 3] += e0 + e1;
-          v[c][j] = pack_bf16(e0, e1);
-        }
-        tmem_st16(s_tmem + c * 16, v[c]);
-      }
-      // The O update is warp-collective (tcgen05.ld/st): run it on the whole warp when any row
-      // needs it. The PV of the previous step completed before S_t was signalled, and the PV of
-      // this step waits for p_full below.
-      if (__any_sync(0xffffffffu, rescale)) {
+      if (turns && lane == 0) mbar_arrive(next_turn);
+      // After a redo the accumulator follows the new reference: O and l scale by alpha. The O
+      // update is warp-collective; the PV of the previous step completed before S_t was
+      // signalled. The first block's PV starts O afresh.
+      if (i > 0 && need_max) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
           tmem_ld32(o_tmem + c * 32, o);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+          for (int jj = 0; jj < 32; ++jj) o[jj] = __float_as_uint(__uint_as_float(o[jj]) * alpha);
           tmem_st32(o_tmem + c * 32, o);
         }
       }
-      l = l * alpha + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
-      m = m_new;
+      l = l * alpha;
+      // P: keys 32c..32c+31 -> packed columns 16c..16c+15 of S_t (S was read before)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_st16(s_tmem + c * 16, v[c]);
+      l += rs;
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full[t]);
       if (tracer) trace_mark(a.trace, 0, role, 4, i);
       __syncwarp();
+      ++i;
     }
+    const int L = i;
     if (ok) {
       if (tracer) trace_mark(a.trace, 0, role, 5, L);
-      if (!warp_wait(&sm.o_done, 0, abort)) {
+      if (!warp_wait(&sm.o_done[t], 0, abort)) {
         fail(sm, a.status, CRISP_ERR_DEVICE_TIMEOUT);
       } else {
         tc_fence_after();
