@@ -61,28 +61,50 @@ __device__ __forceinline__ void fail(AttnSmem& sm, int* status, int code) {
 struct TileList {
   const int32_t* cols;
   int len;
-  __device__ __forceinline__ int at(int i, bool dense, int qb) const {
-    if (dense) return i;
-    const int kb = __ldg(cols + i);
-    return (kb < 0 || kb > qb) ? qb : kb;  // invalid entries are reported and replaced
-  }
 };
 
-// Ascending merge of the two tiles' lists; mask bit t says whether tile t takes part.
+// Ascending merge of the two tiles' lists; mask bit t says whether tile t takes part. Each
+// list's next entry is loaded one step ahead, so its latency hides behind the step. An entry
+// outside [0, qb] or not above its predecessor sets `bad` (the producer reports it) and an
+// out-of-range one is replaced by qb, so every walker stays in bounds and ends after at most
+// len0 + len1 steps; all walkers see the same sequence.
 struct UnionWalk {
   TileList l[2];
-  int i[2];
-  bool dense;
+  int pos[2], head[2], last[2];
+  bool dense, bad;
   int qb;
+  __device__ __forceinline__ UnionWalk(const TileList (&tl)[2], bool dense_, int qb_) : dense(dense_), bad(false), qb(qb_) {
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      l[t] = tl[t];
+      pos[t] = 0;
+      last[t] = -1;
+      head[t] = load(t, 0);
+    }
+  }
+  __device__ __forceinline__ int load(int t, int i) const {
+    if (i >= l[t].len) return 0x7fffffff;
+    return dense ? i : __ldg(l[t].cols + i);
+  }
   __device__ __forceinline__ bool next(int& kb, int& mask) {
-    const bool h0 = i[0] < l[0].len, h1 = i[1] < l[1].len;
-    if (!h0 && !h1) return false;
-    const int a = h0 ? l[0].at(i[0], dense, qb) : 0x7fffffff;
-    const int b = h1 ? l[1].at(i[1], dense, qb) : 0x7fffffff;
-    kb = min(a, b);
-    mask = (a == kb ? 1 : 0) | (b == kb ? 2 : 0);
-    i[0] += mask & 1;
-    i[1] += (mask >> 1) & 1;
+    int h[2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      h[t] = head[t];
+      if (h[t] != 0x7fffffff) {
+        if (h[t] < 0 || h[t] > qb || h[t] <= last[t]) bad = true;
+        if (h[t] < 0 || h[t] > qb) h[t] = qb;
+      }
+    }
+    if (h[0] == 0x7fffffff && h[1] == 0x7fffffff) return false;
+    kb = min(h[0], h[1]);
+    mask = (h[0] == kb ? 1 : 0) | (h[1] == kb ? 2 : 0);
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+      if ((mask >> t) & 1) {
+        last[t] = head[t];
+        head[t] = load(t, ++pos[t]);
+      }
     return true;
   }
 };
@@ -126,7 +148,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int beg = __ldg(rp + qb);
       tl[t].len = __ldg(rp + qb + 1) - beg;
       tl[t].cols = a.cols + (size_t)h * s.cap + beg;
-      bad |= tl[t].len <= 0 || tl[t].len > qb + 1;
+      bad |= tl[t].len <= 0 || tl[t].len > qb + 1 || beg < 0 || (long long)beg + tl[t].len > s.cap;
     }
   }
 
@@ -175,14 +197,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tma_load_2d(&q_map, &sm.q_full, sm.q[t], 0, qrow);
         tma_load_2d(&q_map, &sm.q_full, sm.q[t] + kB * 64, 64, qrow);
       }
-      if (!dense) {
-        for (int t = 0; t < ntiles; ++t)
-          for (int i = 0; i < tl[t].len; ++i) {
-            const int raw = __ldg(tl[t].cols + i);
-            if (raw < 0 || raw > qb) record_status(a.status, CRISP_ERR_DEVICE_CHECK);
-          }
-      }
-      UnionWalk u{{tl[0], tl[1]}, {0, 0}, dense, qb};
+      UnionWalk u(tl, dense, qb);
       int kb, mask, nk = 0;
       for (int step = 0; u.next(kb, mask); ++step) {
         const int st = step % NSK;
@@ -195,6 +210,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tma_load_2d(&k_map, &sm.k_full[st], sm.k[st] + kB * 64, 64, krow);
         nk = step + 1;
       }
+      if (u.bad) record_status(a.status, CRISP_ERR_DEVICE_CHECK);
       // Never leave with copies in flight (bounded waits on the last use of each slot).
       trace_mark(a.trace, 0, 0, 4, 0);
       mbar_wait(&sm.q_full, 0, nullptr);
@@ -207,7 +223,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // Its own thread, so a V slot that is released late never holds back the next K load.
     if (lane == 0) {
       tma_prefetch_desc(&v_map);
-      UnionWalk u{{tl[0], tl[1]}, {0, 0}, dense, qb};
+      UnionWalk u(tl, dense, qb);
       int kb, mask, nv = 0;
       for (int step = 0; u.next(kb, mask); ++step) {
         const int st = step % NSV;
@@ -242,7 +258,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t qa = smem_u32(sm.q[t]);
       bool ok = mbar_wait(&sm.q_full, 0, abort);
       if (!ok) fail(sm, a.status, CRISP_ERR_DEVICE_TIMEOUT);
-      UnionWalk u{{tl[0], tl[1]}, {0, 0}, dense, qb};
+      UnionWalk u(tl, dense, qb);
       int pv_n = 0;  // PV of this tile issued so far
       int prev_mask = 0, kb = 0, mask = 0, step = 0;
       while (ok) {
@@ -321,7 +337,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const bool turns = ntiles == 2;
     uint64_t* my_turn = &sm.turn[t][grp];
     uint64_t* next_turn = &sm.turn[t ^ 1][grp];
-    UnionWalk u{{tl[0], tl[1]}, {0, 0}, dense, qb};
+    UnionWalk u(tl, dense, qb);
     int kb = 0, mask = 0, i = 0;
     for (int j = 0; u.next(kb, mask); ++j) {
       const bool mine = (mask >> t) & 1;

@@ -199,6 +199,51 @@ def test_user_index_through_sparse_prefill():
                                                        [(h, qb) for h in range(hq) for qb in range(nb)], 2))
 
 
+def _dense_index(hq, nb):
+    cap = nb * (nb + 1) // 2
+    row_ptr = np.zeros((hq, nb + 1), dtype=np.int32)
+    cols = np.zeros((hq, cap), dtype=np.int32)
+    for h in range(hq):
+        pos = 0
+        for qb in range(nb):
+            cols[h, pos:pos + qb + 1] = np.arange(qb + 1)
+            pos += qb + 1
+            row_ptr[h, qb + 1] = pos
+    return row_ptr, cols
+
+
+@pytest.mark.parametrize("corrupt", ["out_of_range", "not_ascending", "duplicate", "row_too_long", "row_beyond_cap"])
+def test_malformed_index_is_reported(corrupt):
+    # A malformed user index never reads outside K/V: the kernel reports CRISP_ERR_DEVICE_CHECK.
+    n, hq = 1024, 4
+    q, k, v = (t.to(dev()) for t in W.random_qkv(hq, 2, n, seed=3))
+    nb = n // 128
+    row_ptr, cols = _dense_index(hq, nb)
+    qb = 5
+    beg = row_ptr[3, qb]
+    if corrupt == "out_of_range":
+        cols[3, beg + 2] = 99
+    elif corrupt == "not_ascending":
+        cols[3, beg + 2], cols[3, beg + 3] = cols[3, beg + 3], cols[3, beg + 2]
+    elif corrupt == "duplicate":
+        cols[3, beg + 2] = cols[3, beg + 1]
+    elif corrupt == "row_too_long":
+        row_ptr[3, qb + 1] += 5  # row qb claims more entries than blocks 0..qb
+    else:
+        row_ptr[3, nb] = cols.shape[1] + 3  # last row ends past the head's column array
+    idx = crisp.Index(torch.zeros(hq, dtype=torch.int32, device=dev()), torch.zeros(hq, device=dev()),
+                      torch.from_numpy(row_ptr).to(dev()), torch.from_numpy(cols).to(dev()))
+    ws = crisp.workspace(hq, 2, n, dev())
+    crisp.sparse_prefill(q, k, v, idx, ws=ws)
+    assert crisp.get_status(ws) == -7
+    assert crisp.get_status(ws) == 0  # read and cleared
+    # a head pair without malformed rows is unaffected
+    lists = {0: [list(range(b + 1)) for b in range(nb)]}
+    o, lse = crisp.sparse_prefill(q, k, v, idx, ws=ws)
+    crisp.get_status(ws)
+    PT.assert_attention_ok(PT.compare_attention_blocks(q, k, v, o, lse, lists, [(0, b) for b in range(nb)], 2))
+
+
 def test_bad_arguments_raise():
     q, k, v = (t.to(dev()) for t in W.random_qkv(2, 1, 256, seed=1))
     with pytest.raises(crisp.CrispError):
