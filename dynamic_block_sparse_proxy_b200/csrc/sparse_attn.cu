@@ -13,8 +13,9 @@
 //               write bf16 P back into the tile's S columns; at the end scale O by 1/l, store
 //               bf16 O and the LSE;
 //   warp 8      TMA producer of both Q tiles once, then the K blocks of the union through a
-//               3-stage ring (128-byte swizzle, two 64-column boxes per 128x128 tile);
-//   warp 11     TMA producer of the V blocks through a 2-stage ring;
+//               2-stage ring (128-byte swizzle, two 64-column boxes per 128x128 tile);
+//   warp 11     TMA producer of the V blocks through a 3-stage ring (a V block is consumed a
+//               step after its K block, so it gets the deeper ring);
 //   warps 9-10  one thread per tile issues that tile's UMMAs: O_t += P_t V of the previous step
 //               (A operand read from TMEM), then S_t = Q_t K^T of this step; the two tiles run
 //               out of phase, so the tensor core works on one while the other's softmax runs.
@@ -28,8 +29,8 @@
 namespace crisp {
 namespace {
 
-constexpr int NSK = 3;  // K ring depth
-constexpr int NSV = 2;  // V ring depth
+constexpr int NSK = 2;  // K ring depth
+constexpr int NSV = 3;  // V ring depth (V is consumed a step after K)
 constexpr int THREADS = 384;
 constexpr int PRODUCER_WARP = 8;     // Q and K
 constexpr int V_PRODUCER_WARP = 11;  // V
