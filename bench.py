@@ -14,6 +14,7 @@ bounded sample of the same workload, extrapolated to the same metric.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import subprocess
@@ -110,6 +111,23 @@ def select_bytes(w, n_pe_heads: int, total_pairs: int) -> float:
     qpe = n_pe_heads * w.n * w.d * 2
     idx = 4 * (w.h_q * (nb + 1) + total_pairs)
     return float(k_bytes + qlast + qpe + idx)
+
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attention launch on the 128k
+# workload, from a one-pass ncu capture of this command's own launch. The figure belongs to the
+# kernel source it was taken on; for any other source or workload the bench reports null.
+ATTN_TRAFFIC = {"workload": "llama8b_128k",
+                "source_sha256": "dbf0c5bc3904b8f90c36365e07edbb601bf513b9e713c7b5a2334e35ade98f59",
+                "bytes": 2.73e9 + 1.06e9}
+
+
+def attn_traffic(w):
+    src = os.path.join(ROOT, "dynamic_block_sparse_proxy_b200", "csrc", "sparse_attn.cu")
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    if w.name != ATTN_TRAFFIC["workload"] or sha != ATTN_TRAFFIC["source_sha256"]:
+        return None
+    return ATTN_TRAFFIC["bytes"]
 
 
 def attn_flops(total_pairs: int, d: int = 128) -> float:
@@ -244,7 +262,7 @@ def run_crisp(args):
         "roofline": {"bound": "tensor", "kernel": "sparse_attn", "achieved": achieved_tf,
                      "peak": sustained, "unit": "TFLOP/s", "frac": achieved_tf / sustained,
                      "peak_kind": f"bf16 sustained ({src})",
-                     "frac_of_burst": achieved_tf / pk["bf16_tflops"], "traffic": None,
+                     "frac_of_burst": achieved_tf / pk["bf16_tflops"], "traffic": attn_traffic(w),
                      "flops_per_launch": fl, "selected_pairs": total_pairs,
                      "density": total_pairs / dense_pairs},
         "select_roofline": {"bound": "hbm", "achieved": sel_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
