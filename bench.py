@@ -292,25 +292,29 @@ def oracle_baseline(w, q, k, v, idx, budget_s: float, seed: int = 0) -> dict:
     nb = w.n // 128
     route = idx.route.cpu().numpy() if idx is not None else None
     conc = W.concentrated_heads(w)
-    vs_head = next(h for h in range(w.h_q) if conc[h])
-    pe_head = next(h for h in range(w.h_q) if not conc[h])
+    # one head of each kind the workload has (a one-head workload has only one)
+    vs_head = next((h for h in range(w.h_q) if conc[h]), None)
+    pe_head = next((h for h in range(w.h_q) if not conc[h]), None)
+    heads = [h for h in (vs_head, pe_head) if h is not None]
     f64 = lambda t: t.detach().cpu().to(torch.float64).numpy()  # noqa: E731
     sel, times = {}, {}
-    for h in (vs_head, pe_head):
+    for h in heads:
         qh, kh = f64(q[h]), f64(k[h // G])
         t0 = time.perf_counter()
         sel[h] = O.select_head(qh, kh)
         times[h] = time.perf_counter() - t0
     n_vs = int(route.sum()) if route is not None else sum(conc)
     n_pe = w.h_q - n_vs
-    sel_layer = times[vs_head] * n_vs + times[pe_head] * n_pe
+    t_vs = times[vs_head if vs_head is not None else pe_head]
+    t_pe = times[pe_head if pe_head is not None else vs_head]
+    sel_layer = t_vs * n_vs + t_pe * n_pe
     # attention sample: query blocks of both heads until the budget is used
     rng = np.random.default_rng(seed)
     pairs_done, t_attn = 0, 0.0
     kcache = {}
     start = time.perf_counter()
     while time.perf_counter() - start < budget_s:
-        h = int(rng.choice([vs_head, pe_head]))
+        h = int(rng.choice(heads))
         qb = int(rng.integers(0, nb))
         lists = sel[h]["lists"]
         kv = h // G
@@ -330,8 +334,8 @@ def oracle_baseline(w, q, k, v, idx, budget_s: float, seed: int = 0) -> dict:
     except Exception:
         cores = os.cpu_count() or 1
     return {"value": w.n / layer_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": (f"selection of head {vs_head} (VS) and head {pe_head} (PE) timed in full and "
-                       f"scaled by {n_vs} VS / {n_pe} PE heads; attention on {pairs_done} sampled "
+            "sample": (f"selection of head(s) {heads} (planted-concentrated first) timed in full and "
+                       f"scaled by {n_vs} VS / {n_pe} PE-routed heads; attention on {pairs_done} sampled "
                        f"block pairs ({t_attn:.1f}s) scaled to {total_pairs} selected pairs"),
             "extrapolated_layer_s": layer_s}
 

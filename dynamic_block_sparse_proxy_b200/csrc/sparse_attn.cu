@@ -2,10 +2,11 @@
 // restricted to an index set, softmax(QK^T/sqrt(d) + M_S) V; the CRISP summary's final step,
 // sparse_attention(Q, K, V, S)).
 //
-// One CTA computes one 128-row query block qb for two q-heads of the same GQA group (two
-// "tiles"); both read the same kv-head, so one K/V stream serves both. The CTA walks the union
-// of the two heads' key-block lists in ascending order; a tile takes part in a step only if the
-// block is in its own list.
+// One CTA computes two "tiles", each a 128-row query block of one q-head: the same query block
+// of two q-heads of a GQA group, or (for the last head of an odd group) two adjacent query
+// blocks of one head. Both tiles read the same kv-head, so one K/V stream serves both. The CTA
+// walks the union of the two tiles' key-block lists in ascending order; a tile takes part in a
+// step only if the block is in its own list.
 //   warps 0-3   softmax of tile 0, warps 4-7 softmax of tile 1 (one query row per thread):
 //               read S from TMEM, mask the diagonal block (key j visible to query i iff j <= i),
 //               online softmax in the exp2 domain against a lagging row reference (O and the
@@ -73,11 +74,13 @@ struct UnionWalk {
   TileList l[2];
   int pos[2], head[2], last[2];
   bool dense, bad;
-  int qb;
-  __device__ __forceinline__ UnionWalk(const TileList (&tl)[2], bool dense_, int qb_) : dense(dense_), bad(false), qb(qb_) {
+  int qb[2];
+  __device__ __forceinline__ UnionWalk(const TileList (&tl)[2], bool dense_, const int (&qb_)[2])
+      : dense(dense_), bad(false) {
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
       l[t] = tl[t];
+      qb[t] = qb_[t];
       pos[t] = 0;
       last[t] = -1;
       head[t] = load(t, 0);
@@ -93,8 +96,8 @@ struct UnionWalk {
     for (int t = 0; t < 2; ++t) {
       h[t] = head[t];
       if (h[t] != 0x7fffffff) {
-        if (h[t] < 0 || h[t] > qb || h[t] <= last[t]) bad = true;
-        if (h[t] < 0 || h[t] > qb) h[t] = qb;
+        if (h[t] < 0 || h[t] > qb[t] || h[t] <= last[t]) bad = true;
+        if (h[t] < 0 || h[t] > qb[t]) h[t] = qb[t];
       }
     }
     if (h[0] == 0x7fffffff && h[1] == 0x7fffffff) return false;
@@ -120,23 +123,42 @@ __global__ void __launch_bounds__(THREADS, 1)
   const Shape& s = a.s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // work item: (kv-head, query block, pair of q-heads of its GQA group). kv-heads run one
+  // Work item: two tiles (q-head, query block) that read the same kv-head. kv-heads run one
   // after another and, within one, the longest rows first: the CTAs resident at a time stream
   // the same kv-head's K and V, which then stay in L2 instead of all heads competing for it.
-  const int pairs_per_group = (s.G + 1) / 2;
-  const int per_kv = pairs_per_group * s.nb;
+  // Per kv-head the query blocks go in rows of two (nb-1-2i, nb-2-2i); a row has 2*fp CTAs for
+  // the fp head pairs of the group (one per pair and query block) and, when the group size is
+  // odd, one CTA that takes both query blocks of the group's last head, so no tile runs alone
+  // while another head or block of the same kv-head could share its K/V stream.
+  const int fp = s.G / 2, odd = s.G & 1;
+  const int per_row = 2 * fp + odd;
+  const int per_kv = per_row * ((s.nb + 1) / 2);
   const int kv = (int)(blockIdx.x / per_kv);
   const int rem = (int)(blockIdx.x % per_kv);
-  const int qb = s.nb - 1 - rem / pairs_per_group;
-  const int pig = rem % pairs_per_group;
-  const int h0 = kv * s.G + 2 * pig;
-  const int ntiles = (2 * pig + 1 < s.G) ? 2 : 1;
+  const int row_i = rem / per_row, j = rem % per_row;
+  const int qa = s.nb - 1 - 2 * row_i, qb2 = qa - 1;  // qb2 is -1 past the first query block
+  int tile_h[2], tile_qb[2], ntiles;
+  if (j < 2 * fp) {
+    const int qb = j < fp ? qa : qb2;
+    tile_h[0] = kv * s.G + 2 * (j % fp);
+    tile_h[1] = tile_h[0] + 1;
+    tile_qb[0] = tile_qb[1] = qb;
+    ntiles = qb >= 0 ? 2 : 0;
+  } else {
+    tile_h[0] = tile_h[1] = kv * s.G + s.G - 1;
+    tile_qb[0] = qa;
+    tile_qb[1] = qb2;
+    ntiles = qb2 >= 0 ? 2 : 1;
+  }
+  if (ntiles == 0) return;  // the unpaired half-row when nb is odd: no work
+  if (ntiles == 1) tile_qb[1] = tile_qb[0];
   const bool dense = a.dense != 0;
 
   TileList tl[2];
   bool bad = false;
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
+    const int qb = tile_qb[t];  // t is a compile-time index here (unrolled)
     if (t >= ntiles) {
       tl[t].cols = nullptr;
       tl[t].len = 0;
@@ -144,7 +166,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tl[t].cols = nullptr;
       tl[t].len = qb + 1;
     } else {
-      const int h = h0 + t;
+      const int h = tile_h[t];
       const int32_t* rp = a.row_ptr + (size_t)h * (s.nb + 1);
       const int beg = __ldg(rp + qb);
       tl[t].len = __ldg(rp + qb + 1) - beg;
@@ -194,11 +216,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       tma_prefetch_desc(&k_map);
       mbar_arrive_expect_tx(&sm.q_full, TILE_BYTES * ntiles);
       for (int t = 0; t < ntiles; ++t) {
-        const int qrow = (h0 + t) * s.n + qb * kB;
+        const int qrow = (t ? tile_h[1] : tile_h[0]) * s.n + (t ? tile_qb[1] : tile_qb[0]) * kB;
         tma_load_2d(&q_map, &sm.q_full, sm.q[t], 0, qrow);
         tma_load_2d(&q_map, &sm.q_full, sm.q[t] + kB * 64, 64, qrow);
       }
-      UnionWalk u(tl, dense, qb);
+      UnionWalk u(tl, dense, tile_qb);
       int kb, mask, nk = 0;
       for (int step = 0; u.next(kb, mask); ++step) {
         const int st = step % NSK;
@@ -224,7 +246,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // Its own thread, so a V slot that is released late never holds back the next K load.
     if (lane == 0) {
       tma_prefetch_desc(&v_map);
-      UnionWalk u(tl, dense, qb);
+      UnionWalk u(tl, dense, tile_qb);
       int kb, mask, nv = 0;
       for (int step = 0; u.next(kb, mask); ++step) {
         const int st = step % NSV;
@@ -259,7 +281,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t qa = smem_u32(sm.q[t]);
       bool ok = mbar_wait(&sm.q_full, 0, abort);
       if (!ok) fail(sm, a.status, CRISP_ERR_DEVICE_TIMEOUT);
-      UnionWalk u(tl, dense, qb);
+      UnionWalk u(tl, dense, tile_qb);
       int pv_n = 0;  // PV of this tile issued so far
       int prev_mask = 0, kb = 0, mask = 0, step = 0;
       while (ok) {
@@ -322,6 +344,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp < 4 * ntiles) {
     // ------------------------------------------------------------------ softmax + epilogue
     const int t = warp >> 2;
+    const int my_qb = t ? tile_qb[1] : tile_qb[0];
+    const int my_h = t ? tile_h[1] : tile_h[0];
     const int grp = warp & 3;
     const int r = grp * 32 + lane;
     const int role = 2 + t;                     // traced by the first warp of each tile
@@ -338,7 +362,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const bool turns = ntiles == 2;
     uint64_t* my_turn = &sm.turn[t][grp];
     uint64_t* next_turn = &sm.turn[t ^ 1][grp];
-    UnionWalk u(tl, dense, qb);
+    UnionWalk u(tl, dense, tile_qb);
     int kb = 0, mask = 0, i = 0;
     for (int j = 0; u.next(kb, mask); ++j) {
       const bool mine = (mask >> t) & 1;
@@ -376,7 +400,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           turn_ok = false;
           break;
         }
-        if (kb == qb) {
+        if (kb == my_qb) {
 #pragma unroll
           for (int c = 0; c < 4; ++c)
 #pragma unroll
@@ -454,8 +478,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       } else {
         tc_fence_after();
         const float inv = 1.f / l;
-        const int h = h0 + t;
-        const size_t row = (size_t)h * s.n + (size_t)qb * kB + r;
+        const size_t row = (size_t)my_h * s.n + (size_t)my_qb * kB + r;
         uint4* dst = reinterpret_cast<uint4*>(a.o + row * kD);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -495,8 +518,9 @@ cudaError_t launch_sparse_attn(const CUtensorMap& q_map, const CUtensorMap& k_ma
   cudaError_t e =
       cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int n_pairs = a.s.h_kv * ((a.s.G + 1) / 2);
-  sparse_attn_kernel<<<n_pairs * a.s.nb, THREADS, smem, st>>>(q_map, k_map, v_map, a);
+  const int per_row = 2 * (a.s.G / 2) + (a.s.G & 1);
+  const int grid = a.s.h_kv * per_row * ((a.s.nb + 1) / 2);
+  sparse_attn_kernel<<<grid, THREADS, smem, st>>>(q_map, k_map, v_map, a);
   return cudaGetLastError();
 }
 

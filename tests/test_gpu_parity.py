@@ -64,7 +64,7 @@ def test_timeout_selftest_reports_and_context_survives():
     assert np.max(np.abs(PT.f64(o[0]) - ref)) < 2e-2
 
 
-@pytest.mark.parametrize("n,hq,hkv", [(128, 1, 1), (256, 2, 1), (640, 3, 1), (1024, 4, 2)])
+@pytest.mark.parametrize("n,hq,hkv", [(128, 1, 1), (256, 2, 1), (384, 1, 1), (640, 3, 1), (896, 7, 1), (1024, 4, 2)])
 def test_dense_matches_oracle(n, hq, hkv):
     q, k, v = (t.to(dev()) for t in W.random_qkv(hq, hkv, n, seed=n + hq))
     ws = crisp.workspace(hq, hkv, n, dev())
@@ -172,9 +172,11 @@ def test_pe_uniform_closed_form_on_gpu():
         assert idx.lists(h) == [x.tolist() for x in sels[h]["lists"]]
 
 
-def test_user_index_through_sparse_prefill():
-    n, hq = 2048, 4
-    q, k, v = (t.to(dev()) for t in W.random_qkv(hq, 2, n, seed=5))
+@pytest.mark.parametrize("n,hq,hkv", [(2048, 4, 2), (1152, 3, 1), (640, 1, 1), (1920, 14, 2)])
+def test_user_index_through_sparse_prefill(n, hq, hkv):
+    # random strictly ascending lists with the diagonal block; odd group sizes and odd block
+    # counts pair a head's adjacent query blocks in one CTA
+    q, k, v = (t.to(dev()) for t in W.random_qkv(hq, hkv, n, seed=5))
     nb = n // 128
     rng = np.random.default_rng(9)
     cap = nb * (nb + 1) // 2
@@ -192,11 +194,11 @@ def test_user_index_through_sparse_prefill():
             row_ptr[h, qb + 1] = pos
     idx = crisp.Index(torch.zeros(hq, dtype=torch.int32, device=dev()), torch.zeros(hq, device=dev()),
                       torch.from_numpy(row_ptr).to(dev()), torch.from_numpy(cols).to(dev()))
-    ws = crisp.workspace(hq, 2, n, dev())
+    ws = crisp.workspace(hq, hkv, n, dev())
     o, lse = crisp.sparse_prefill(q, k, v, idx, ws=ws)
     crisp.check_status(ws)
     PT.assert_attention_ok(PT.compare_attention_blocks(q, k, v, o, lse, lists,
-                                                       [(h, qb) for h in range(hq) for qb in range(nb)], 2))
+                                                       [(h, qb) for h in range(hq) for qb in range(nb)], hq // hkv))
 
 
 def _dense_index(hq, nb):
