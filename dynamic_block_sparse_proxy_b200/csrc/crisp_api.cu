@@ -139,13 +139,15 @@ int run_select(const void* q, const void* k, const Shape& s, const crisp_params*
 }
 
 int run_attention(const void* q, const void* k, const void* v, const Shape& s, const int32_t* row_ptr,
-                  const int32_t* cols, int dense, void* o, float* lse, void* ws, cudaStream_t st) {
+                  const int32_t* cols, const int32_t* route, int dense, void* o, float* lse, void* ws,
+                  cudaStream_t st) {
   const Workspace w = workspace_layout(s);
   AttnArgs a{};
   a.s = s;
   a.dense = dense;
   a.row_ptr = row_ptr;
   a.cols = cols;
+  a.route = route;
   a.o = static_cast<__nv_bfloat16*>(o);
   a.lse = lse;
   a.status = at<int>(ws, w.status);
@@ -214,7 +216,8 @@ int crisp_sparse_prefill(const void* q, const void* k, const void* v, int h_q, i
   if (rc == CRISP_OK) rc = check_index(idx, false);
   if (rc == CRISP_OK) rc = check_ws(ws, ws_bytes, s);
   if (rc != CRISP_OK) return rc;
-  return run_attention(q, k, v, s, idx->row_ptr, idx->cols, 0, o, lse, ws, static_cast<cudaStream_t>(stream));
+  return run_attention(q, k, v, s, idx->row_ptr, idx->cols, idx->route, 0, o, lse, ws,
+                       static_cast<cudaStream_t>(stream));
 }
 
 int crisp_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv, int n, int d,
@@ -242,7 +245,7 @@ int crisp_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   rc = run_select(q, k, s, params, idx, ws, st);
   if (rc != CRISP_OK) return rc;
-  return run_attention(q, k, v, s, idx.row_ptr, idx.cols, 0, o, lse, ws, st);
+  return run_attention(q, k, v, s, idx.row_ptr, idx.cols, idx.route, 0, o, lse, ws, st);
 }
 
 int crisp_dense_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv, int n, int d, void* o,
@@ -253,7 +256,7 @@ int crisp_dense_prefill(const void* q, const void* k, const void* v, int h_q, in
     rc = CRISP_ERR_INVALID_ARG;
   if (rc == CRISP_OK) rc = check_ws(ws, ws_bytes, s);
   if (rc != CRISP_OK) return rc;
-  return run_attention(q, k, v, s, nullptr, nullptr, 1, o, lse, ws, static_cast<cudaStream_t>(stream));
+  return run_attention(q, k, v, s, nullptr, nullptr, nullptr, 1, o, lse, ws, static_cast<cudaStream_t>(stream));
 }
 
 int crisp_get_status(void* ws, void* stream) {

@@ -117,6 +117,7 @@ struct AttnArgs {
   int dense;             // 1: every block <= qb, index ignored
   const int32_t* row_ptr;
   const int32_t* cols;
+  const int32_t* route;  // per q-head class used to pair heads in a CTA; may be null
   __nv_bfloat16* o;
   float* lse;
   int* status;

@@ -3,8 +3,8 @@
 // sparse_attention(Q, K, V, S)).
 //
 // One CTA computes two "tiles", each a 128-row query block of one q-head: the same query block
-// of two q-heads of a GQA group, or (for the last head of an odd group) two adjacent query
-// blocks of one head. Both tiles read the same kv-head, so one K/V stream serves both. The CTA
+// of two q-heads of a GQA group that were routed alike, or two adjacent query blocks of one
+// head. Both tiles read the same kv-head, so one K/V stream serves both. The CTA
 // walks the union of the two tiles' key-block lists in ascending order; a tile takes part in a
 // step only if the block is in its own list.
 //   warps 0-3   softmax of tile 0, warps 4-7 softmax of tile 1 (one query row per thread):
@@ -126,29 +126,52 @@ __global__ void __launch_bounds__(THREADS, 1)
   // Work item: two tiles (q-head, query block) that read the same kv-head. kv-heads run one
   // after another and, within one, the longest rows first: the CTAs resident at a time stream
   // the same kv-head's K and V, which then stay in L2 instead of all heads competing for it.
-  // Per kv-head the query blocks go in rows of two (nb-1-2i, nb-2-2i); a row has 2*fp CTAs for
-  // the fp head pairs of the group (one per pair and query block) and, when the group size is
-  // odd, one CTA that takes both query blocks of the group's last head, so no tile runs alone
-  // while another head or block of the same kv-head could share its K/V stream.
-  const int fp = s.G / 2, odd = s.G & 1;
-  const int per_row = 2 * fp + odd;
-  const int per_kv = per_row * ((s.nb + 1) / 2);
+  // Per kv-head the query blocks go in rows of two (qa = nb-1-2i, qa-1), G CTAs per row. The
+  // group's heads are taken Vertical-Slash first, then Pooled-Estimation (by `route`, when
+  // given), each in ascending order; consecutive heads of one class form a pair that gets two
+  // CTAs (one per query block), and a class's leftover head gets one CTA holding both of its
+  // query blocks. Heads of one class select alike, so a CTA's two lists overlap and most steps
+  // feed both tiles; either way the G heads fill exactly G slots per row.
+  const int per_kv = s.G * ((s.nb + 1) / 2);
   const int kv = (int)(blockIdx.x / per_kv);
   const int rem = (int)(blockIdx.x % per_kv);
-  const int row_i = rem / per_row, j = rem % per_row;
-  const int qa = s.nb - 1 - 2 * row_i, qb2 = qa - 1;  // qb2 is -1 past the first query block
-  int tile_h[2], tile_qb[2], ntiles;
-  if (j < 2 * fp) {
-    const int qb = j < fp ? qa : qb2;
-    tile_h[0] = kv * s.G + 2 * (j % fp);
-    tile_h[1] = tile_h[0] + 1;
-    tile_qb[0] = tile_qb[1] = qb;
-    ntiles = qb >= 0 ? 2 : 0;
-  } else {
-    tile_h[0] = tile_h[1] = kv * s.G + s.G - 1;
-    tile_qb[0] = qa;
-    tile_qb[1] = qb2;
-    ntiles = qb2 >= 0 ? 2 : 1;
+  const int row_i = rem / s.G, slot = rem % s.G;
+  const int qa = s.nb - 1 - 2 * row_i;  // qa - 1 is -1 past the first query block
+  int tile_h[2] = {0, 0}, tile_qb[2] = {qa, qa}, ntiles = 0;
+  {
+    int next_slot = 0, pending = -1;
+    bool found = false;
+    for (int cls = 1; cls >= 0 && !found; --cls) {
+      for (int x = 0; x < s.G && !found; ++x) {
+        const int h = kv * s.G + x;
+        const int c = a.route != nullptr ? (__ldg(a.route + h) != 0 ? 1 : 0) : 1;
+        if (c != cls) continue;
+        if (pending < 0) {
+          pending = h;
+          continue;
+        }
+        if (slot == next_slot || slot == next_slot + 1) {  // head pair, one query block each
+          tile_h[0] = pending;
+          tile_h[1] = h;
+          tile_qb[0] = tile_qb[1] = qa - (slot - next_slot);
+          ntiles = tile_qb[0] >= 0 ? 2 : 0;
+          found = true;
+        }
+        next_slot += 2;
+        pending = -1;
+      }
+      if (!found && pending >= 0) {
+        if (slot == next_slot) {  // leftover head: two adjacent query blocks of it
+          tile_h[0] = tile_h[1] = pending;
+          tile_qb[0] = qa;
+          tile_qb[1] = qa - 1;
+          ntiles = qa - 1 >= 0 ? 2 : 1;
+          found = true;
+        }
+        next_slot += 1;
+        pending = -1;
+      }
+    }
   }
   if (ntiles == 0) return;  // the unpaired half-row when nb is odd: no work
   if (ntiles == 1) tile_qb[1] = tile_qb[0];
@@ -518,8 +541,7 @@ cudaError_t launch_sparse_attn(const CUtensorMap& q_map, const CUtensorMap& k_ma
   cudaError_t e =
       cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int per_row = 2 * (a.s.G / 2) + (a.s.G & 1);
-  const int grid = a.s.h_kv * per_row * ((a.s.nb + 1) / 2);
+  const int grid = a.s.h_q * ((a.s.nb + 1) / 2);
   sparse_attn_kernel<<<grid, THREADS, smem, st>>>(q_map, k_map, v_map, a);
   return cudaGetLastError();
 }

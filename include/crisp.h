@@ -102,7 +102,11 @@ int crisp_select(const void* q, const void* k, int h_q, int h_kv, int n, int d,
 /*
  * Block-sparse causal attention (CRISP §2: softmax(QK^T/sqrt(d) + M_S) V with M_S = 0 on the
  * selected blocks and -inf elsewhere; within a block, key j is visible to query i iff j <= i).
- * Reads idx->row_ptr and idx->cols; every row must contain at least one block <= qb.
+ * Reads idx->row_ptr and idx->cols; every row must contain at least one block <= qb. A row
+ * that is empty, longer than qb+1, outside the head's column array, not strictly ascending or
+ * holding a block outside [0, qb] is reported as CRISP_ERR_DEVICE_CHECK (crisp_get_status) and
+ * never read out of bounds. idx->route may be NULL; when given, heads of one GQA group with the
+ * same route (any non-zero value counts as 1) are scheduled together. It only affects speed.
  * o: bf16 [h_q][n][d]. lse: fp32 [h_q][n] natural-log sum-exp of the scaled logits, or NULL.
  */
 int crisp_sparse_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv, int n,

@@ -172,8 +172,9 @@ def test_pe_uniform_closed_form_on_gpu():
         assert idx.lists(h) == [x.tolist() for x in sels[h]["lists"]]
 
 
-@pytest.mark.parametrize("n,hq,hkv", [(2048, 4, 2), (1152, 3, 1), (640, 1, 1), (1920, 14, 2)])
-def test_user_index_through_sparse_prefill(n, hq, hkv):
+@pytest.mark.parametrize("n,hq,hkv,mixed", [(2048, 4, 2, False), (1152, 3, 1, False), (640, 1, 1, False),
+                                            (1920, 14, 2, True), (1152, 5, 1, True)])
+def test_user_index_through_sparse_prefill(n, hq, hkv, mixed):
     # random strictly ascending lists with the diagonal block; odd group sizes and odd block
     # counts pair a head's adjacent query blocks in one CTA
     q, k, v = (t.to(dev()) for t in W.random_qkv(hq, hkv, n, seed=5))
@@ -192,7 +193,9 @@ def test_user_index_through_sparse_prefill(n, hq, hkv):
             cols[h, pos:pos + len(sel)] = sel
             pos += len(sel)
             row_ptr[h, qb + 1] = pos
-    idx = crisp.Index(torch.zeros(hq, dtype=torch.int32, device=dev()), torch.zeros(hq, device=dev()),
+    # a mixed route splits each group into classes that are scheduled apart
+    route = torch.from_numpy(rng.integers(0, 2, size=hq).astype(np.int32)) if mixed else torch.zeros(hq, dtype=torch.int32)
+    idx = crisp.Index(route.to(dev()), torch.zeros(hq, device=dev()),
                       torch.from_numpy(row_ptr).to(dev()), torch.from_numpy(cols).to(dev()))
     ws = crisp.workspace(hq, hkv, n, dev())
     o, lse = crisp.sparse_prefill(q, k, v, idx, ws=ws)
