@@ -67,18 +67,24 @@ __device__ int block_argmax(double v, int idx, double* redv, int* redi) {
 
 // 1. Per proxy row r of head h: global reference max M_r over the chunks, normaliser Z_r, and
 //    the weight w = exp2(m_chunk - M_r) / (Z_r * B) that turns a chunk's sums into column-mean mass.
-__global__ void __launch_bounds__(kB) row_stats_kernel(const SelectArgs a) {
+//    One warp per row, its lanes across the chunks.
+constexpr int STAT_ROWS = 8;
+__global__ void __launch_bounds__(STAT_ROWS * 32) row_stats_kernel(const SelectArgs a) {
   const Shape& s = a.s;
-  const int h = blockIdx.x, r = threadIdx.x;
+  const int h = blockIdx.y, r = blockIdx.x * STAT_ROWS + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   const float* mc = a.chunk_max + (size_t)h * s.n_chunks * kB;
   const float* tc = a.chunk_tot + (size_t)h * s.n_chunks * kB;
   float M = -INFINITY;
-  for (int c = 0; c < s.n_chunks; ++c) M = fmaxf(M, mc[c * kB + r]);
+  for (int c = lane; c < s.n_chunks; c += 32) M = fmaxf(M, mc[c * kB + r]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   double Z = 0.0;
-  for (int c = 0; c < s.n_chunks; ++c) Z += (double)exp2f(mc[c * kB + r] - M) * (double)tc[c * kB + r];
+  for (int c = lane; c < s.n_chunks; c += 32) Z += (double)exp2f(mc[c * kB + r] - M) * (double)tc[c * kB + r];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, o);
   float* w = a.row_w + (size_t)h * s.n_chunks * kB;
   const double inv = 1.0 / (Z * kB);
-  for (int c = 0; c < s.n_chunks; ++c) w[c * kB + r] = (float)((double)exp2f(mc[c * kB + r] - M) * inv);
+  for (int c = lane; c < s.n_chunks; c += 32) w[c * kB + r] = (float)((double)exp2f(mc[c * kB + r] - M) * inv);
 }
 
 // 2. Block masses, one warp per key block: p_v[kb] = sum_r w*(lo+hi); the lower-offset halves
@@ -208,7 +214,7 @@ __global__ void __launch_bounds__(THREADS) route_threshold_kernel(const SelectAr
 }  // namespace
 
 cudaError_t launch_route_threshold(const SelectArgs& a, cudaStream_t st) {
-  row_stats_kernel<<<a.s.h_q, kB, 0, st>>>(a);
+  row_stats_kernel<<<dim3(kB / STAT_ROWS, a.s.h_q), STAT_ROWS * 32, 0, st>>>(a);
   block_mass_kernel<<<dim3((a.s.nb + MASS_WARPS - 1) / MASS_WARPS, a.s.h_q), MASS_WARPS * 32, 0, st>>>(a);
   const size_t smem = (size_t)2 * a.s.nb * sizeof(double);
   cudaError_t e = cudaFuncSetAttribute(route_threshold_kernel,
