@@ -28,6 +28,14 @@ Readings where the pages leave a step open (each also listed in the design notes
   R7 the PE gamma cut is one global cut over the flattened block-causal pooled matrix
      (total mass N_b), order (P desc, qb asc, kb asc), shortest prefix with cumsum >= gamma*N_b;
      every PE row also keeps {0, qb-1, qb}; gamma >= 1 keeps everything.
+  R8 (FlexPrefill baseline, [CRISP] §2 and §3 discussion) the pooled estimate a_bar is the
+     softmax over all N_b key blocks of mean(Q_last) . Kbar[kb] / sqrt(d); the per-query mean
+     a_hat pooled to blocks is p_v; JSD uses natural logs (0 log 0 = 0); VS iff JSD >= tau;
+  R9 (FlexPrefill baseline) each direction keeps the shortest prefix of its blocks sorted
+     (p desc, index asc) whose sum reaches gamma times the direction's total; the first and last
+     blocks are added as for CRISP (the merge of R6 is unchanged);
+  R10 (median floor, [CRISP] §4 robustness discussion / Table 9) mu_d is the median of
+     p_d[1..N_b-2] (mean of the two middle values when N_b-2 is even); the keep rule is unchanged.
 """
 from __future__ import annotations
 
@@ -68,6 +76,23 @@ def route_is_vs(c: float, tau: float) -> bool:
     return c >= tau
 
 
+def pooled_estimate(q_last: np.ndarray, k: np.ndarray, B: int) -> np.ndarray:
+    """FlexPrefill's a_bar: softmax over all key blocks of mean(q_last) . Kbar[kb] / sqrt(d) (R8)."""
+    d = q_last.shape[1]
+    s = (q_last.mean(axis=0) @ block_mean(k, B).T) / np.sqrt(d)
+    e = np.exp(s - s.max())
+    return e / e.sum()
+
+
+def jsd(p: np.ndarray, q: np.ndarray) -> float:
+    """Jensen-Shannon divergence (natural log): KL(p||m)/2 + KL(q||m)/2 with m = (p+q)/2."""
+    m = 0.5 * (p + q)
+    def kl(a):
+        nz = a > 0
+        return float(np.sum(a[nz] * np.log(a[nz] / m[nz])))
+    return 0.5 * kl(p) + 0.5 * kl(q)
+
+
 # ----------------------------------------------------------------------------------------------
 # Vertical and slash scores pooled into key blocks  ([CRISP] §4, decomposition paragraph)
 # ----------------------------------------------------------------------------------------------
@@ -100,11 +125,35 @@ def noise_floor(p: np.ndarray) -> float:
     return max(1.0 - p[0] - p[-1], 0.0) / (nb - 2)
 
 
-def keep_blocks(p: np.ndarray, alpha: float, min_blocks: int = 0) -> list[int]:
-    """Blocks j in [1, N_b-2] with p[j] > alpha*mu (strict), topped up to min_blocks (R5)."""
+def median_floor(p: np.ndarray) -> float:
+    """mu = median of the non-anchor block masses p[1..N_b-2] (R10)."""
+    return float(np.median(p[1:-1]))
+
+
+def gamma_keep_direction(p: np.ndarray, gamma: float) -> tuple[list[int], float]:
+    """FlexPrefill's per-direction rule (R9): the shortest prefix of the blocks sorted (p desc,
+    j asc) whose sum reaches gamma * sum(p). Returns (kept blocks in [1, N_b-2], cut value)."""
     nb = p.shape[0]
-    mu = noise_floor(p)
+    order = np.lexsort((np.arange(nb), -p))
+    csum = np.cumsum(p[order])
+    hit = np.nonzero(csum >= gamma * p.sum())[0]
+    count = int(hit[0]) + 1 if hit.size else nb
+    kept = order[:count]
+    return sorted(int(j) for j in kept if 1 <= j <= nb - 2), float(p[order[count - 1]])
+
+
+def keep_blocks(p: np.ndarray, alpha: float, min_blocks: int = 0, floor: str = "mean") -> list[int]:
+    """Blocks j in [1, N_b-2] with p[j] > alpha*mu (strict), topped up to min_blocks (R5);
+    mu is the mean floor of [CRISP] §4 or the median floor (R10)."""
+    nb = p.shape[0]
+    mu = noise_floor(p) if floor == "mean" else median_floor(p)
     keep = [j for j in range(1, nb - 1) if p[j] > alpha * mu]
+    return top_up(p, keep, min_blocks)
+
+
+def top_up(p: np.ndarray, keep: list[int], min_blocks: int) -> list[int]:
+    """Add the largest remaining blocks of [1, N_b-2] (ties: lower index) up to min_blocks (R5)."""
+    nb = p.shape[0]
     if min_blocks > len(keep):
         rest = [j for j in range(1, nb - 1) if j not in set(keep)]
         rest.sort(key=lambda j: (-p[j], j))
@@ -201,11 +250,17 @@ def pe_select(q: np.ndarray, k: np.ndarray, B: int, gamma: float):
 # ----------------------------------------------------------------------------------------------
 # Per-head selection  ([BLOG] per-head flow; [CRISP] §3.2, §4)
 # ----------------------------------------------------------------------------------------------
+JSD_TIE_REL = 1e-4  # routing band of the JSD rule: a_bar comes from fp32 pooled means
+
+
 def select_head(q: np.ndarray, k: np.ndarray, *, block=128, anchors=128, tau_proxy=0.5,
-                alpha=1.0, gamma=0.95, min_blocks=0) -> dict:
+                alpha=1.0, gamma=0.95, min_blocks=0, route_rule="cstruct", tau_jsd=0.1,
+                vs_rule="floor", floor="mean") -> dict:
     """Route one q-head and build its per-query-block key-block lists.
 
     q: [n, d] fp64 queries of the head; k: [n, d] fp64 keys of its kv-head.
+    CRISP: route_rule="cstruct", vs_rule="floor" (floor="mean", or "median" for R10).
+    FlexPrefill baseline: route_rule="jsd" (R8), vs_rule="gamma" (R9).
     """
     n = q.shape[0]
     B = block
@@ -214,18 +269,41 @@ def select_head(q: np.ndarray, k: np.ndarray, *, block=128, anchors=128, tau_pro
     c = c_struct(a_hat, n, anchors)
     p_v = vertical_block_mass(a_hat, B)
     p_s = slash_block_mass(a_hat, n, B)
-    vs = route_is_vs(c, tau_proxy)
-    out = dict(c_struct=c, route=int(vs), p_v=p_v, p_s=p_s, route_tie=abs(c - tau_proxy) <= TIE_REL * tau_proxy)
+    out = dict(c_struct=c, p_v=p_v, p_s=p_s)
+    if route_rule == "jsd":
+        j = jsd(pooled_estimate(q[n - B:], k, B), p_v)
+        vs = j >= tau_jsd
+        out.update(jsd=j, route_tie=abs(j - tau_jsd) <= JSD_TIE_REL * max(tau_jsd, j))
+    else:
+        vs = route_is_vs(c, tau_proxy)
+        out["route_tie"] = abs(c - tau_proxy) <= TIE_REL * tau_proxy
+    out["route"] = int(vs)
     if nb >= 3:
-        out["mu_v"], out["mu_s"] = noise_floor(p_v), noise_floor(p_s)
+        if floor == "median":
+            out["mu_v"], out["mu_s"] = median_floor(p_v), median_floor(p_s)
+        else:
+            out["mu_v"], out["mu_s"] = noise_floor(p_v), noise_floor(p_s)
     if vs:
         if nb <= 2:
             out["lists"] = [np.arange(qb + 1) for qb in range(nb)]
             out["keep_v"], out["keep_s"] = [], []
             out["vs_ties_v"], out["vs_ties_s"] = [], []
+        elif vs_rule == "gamma":
+            for name, p in (("v", p_v), ("s", p_s)):
+                kept, cut = gamma_keep_direction(p, gamma)
+                out["keep_" + name] = top_up(p, kept, min_blocks)
+                # ties: values within TIE_REL of the cut value, or a prefix sum within TIE_REL of
+                # the target (either can flip with rounding)
+                order = np.lexsort((np.arange(nb), -p))
+                before = np.cumsum(p[order]) - p[order]
+                target = gamma * p.sum()
+                near = set(int(order[i]) for i in range(nb) if abs(before[i] - target) <= TIE_REL * target)
+                near |= {jj for jj in range(nb) if abs(p[jj] - cut) <= TIE_REL * cut}
+                out["vs_ties_" + name] = sorted(jj for jj in near if 1 <= jj <= nb - 2)
+            out["lists"] = merge_vertical_slash(out["keep_v"], out["keep_s"], nb)
         else:
-            keep_v = keep_blocks(p_v, alpha, min_blocks)
-            keep_s = keep_blocks(p_s, alpha, min_blocks)
+            keep_v = keep_blocks(p_v, alpha, min_blocks, floor)
+            keep_s = keep_blocks(p_s, alpha, min_blocks, floor)
             out["keep_v"], out["keep_s"] = keep_v, keep_s
             out["lists"] = merge_vertical_slash(keep_v, keep_s, nb)
             for name, p, mu in (("v", p_v, out["mu_v"]), ("s", p_s, out["mu_s"])):

@@ -360,3 +360,84 @@ def test_qwen_geometry_sink_dominates_concentrated_heads():
         assert s["route"] == int(meta["concentrated"][h])
         if meta["concentrated"][h]:
             assert s["p_v"][0] > 0.9
+
+
+# ------------------------------------------------------------------ FlexPrefill rules, median floor
+def test_jsd_closed_forms():
+    p = np.array([0.2, 0.3, 0.5])
+    assert O.jsd(p, p) == 0.0
+    # disjoint supports: ln 2 (natural log)
+    assert math.isclose(O.jsd(np.array([1.0, 0.0]), np.array([0.0, 1.0])), math.log(2.0), rel_tol=1e-15)
+    # hand value: p = (1, 0), q = (1/2, 1/2), m = (3/4, 1/4)
+    # KL(p||m) = ln(4/3); KL(q||m) = (1/2) ln(2/3) + (1/2) ln 2
+    want = 0.5 * math.log(4 / 3) + 0.5 * (0.5 * math.log(2 / 3) + 0.5 * math.log(2.0))
+    assert math.isclose(O.jsd(np.array([1.0, 0.0]), np.array([0.5, 0.5])), want, rel_tol=1e-14)
+    rng = np.random.default_rng(1)
+    a, b = rng.random(7), rng.random(7)
+    a, b = a / a.sum(), b / b.sum()
+    assert math.isclose(O.jsd(a, b), O.jsd(b, a), rel_tol=1e-14)
+    assert 0.0 < O.jsd(a, b) < math.log(2.0)
+
+
+def test_pooled_estimate_hand_case():
+    # d = 2, B = 2: mean query (sqrt(2) ln 3, 0) against block means (1, 0) and (0, 1) gives
+    # logits (ln 3, 0) after the 1/sqrt(d) scale, i.e. a_bar = (3/4, 1/4)
+    qbar = np.array([math.sqrt(2.0) * math.log(3.0), 0.0])
+    q_last = np.stack([qbar + [0.5, -1.0], qbar - [0.5, -1.0]])   # mean is qbar
+    k = np.array([[1.0, 0.0], [1.0, 0.0], [0.0, 1.0], [0.0, 1.0]])
+    np.testing.assert_allclose(O.pooled_estimate(q_last, k, 2), [0.75, 0.25], rtol=1e-14)
+    # identical key blocks: uniform
+    np.testing.assert_allclose(O.pooled_estimate(q_last, np.ones((6, 2)), 2), np.full(3, 1 / 3), rtol=1e-14)
+
+
+def test_gamma_keep_direction_hand_cases():
+    p = np.array([0.5, 0.1, 0.3, 0.1])
+    assert O.gamma_keep_direction(p, 0.8) == ([2], 0.3)         # {0, 2} reach 0.8; 0 is an anchor
+    assert O.gamma_keep_direction(p, 0.85) == ([1, 2], 0.1)     # the tie at 0.1 goes to j=1 first
+    assert O.gamma_keep_direction(p, 0.95) == ([1, 2], 0.1)     # 0.1 at j=3 only comes after
+    assert O.gamma_keep_direction(p, 1.0)[0] == [1, 2]
+    # a target scaled by the direction's own total
+    assert O.gamma_keep_direction(2 * p, 0.8) == ([2], 0.6)
+
+
+def test_median_floor_and_keep():
+    p = np.array([0.4, 0.1, 0.3, 0.05, 0.15])                   # inner 0.1, 0.3, 0.05 -> 0.1
+    assert O.median_floor(p) == 0.1
+    assert O.keep_blocks(p, 1.0, floor="median") == [2]
+    assert O.keep_blocks(p, 0.4, floor="median") == [1, 2, 3]   # 0.05 > 0.04
+    q = np.array([0.5, 0.1, 0.2, 0.04, 0.06, 0.1])              # inner even: (0.06 + 0.1) / 2
+    assert math.isclose(O.median_floor(q), 0.08, rel_tol=1e-15)
+    # the mean floor of the same inner mass differs: (1 - 0.5 - 0.1) / 4 = 0.1
+    assert math.isclose(O.noise_floor(q), 0.1, rel_tol=1e-14)
+    assert O.keep_blocks(q, 1.0, floor="median") == [1, 2]       # j = 5 is the last anchor
+    assert O.keep_blocks(q, 1.0, floor="mean") == [2]
+
+
+def test_flexprefill_rules_on_planted_heads():
+    """JSD is large on planted-concentrated heads and small on diffuse ones. On a sink-dominated
+    head the per-direction gamma cut stops at the sink block (the mass-cliff collapse the CRISP
+    paper describes, §4), so no inner vertical block survives; gamma = 1 keeps every block that
+    carries mass."""
+    w = W.WORKLOADS["llama8b_32k"].scaled(4096)
+    q, k, v, meta = W.generate(w)
+    G = w.h_q // w.h_kv
+    nb = w.n // 128
+    for h in (0, 2):
+        s = O.select_head(q[h].double().numpy(), k[h // G].double().numpy(), route_rule="jsd",
+                          vs_rule="gamma")
+        assert s["route"] == int(meta["concentrated"][h]), s["jsd"]
+        if s["route"]:
+            assert s["jsd"] > 0.3
+            assert s["p_v"][0] >= 0.95 and s["keep_v"] == []
+        else:
+            assert s["jsd"] < 0.01
+    s = O.select_head(q[0].double().numpy(), k[0].double().numpy(), route_rule="jsd", vs_rule="gamma",
+                      gamma=1.0)
+    assert s["keep_v"] == [j for j in range(1, nb - 1) if s["p_v"][j] > 0]
+    # with a target below the sink's share but above it plus the planted blocks' mass, the
+    # planted verticals come first among the inner blocks
+    pv = s["p_v"]
+    inner_planted = sorted(meta["vertical_blocks"][0])
+    g = (pv[0] + pv[nb - 1] + pv[inner_planted].sum() * 0.999) / pv.sum()
+    kept, _ = O.gamma_keep_direction(pv, g)
+    assert set(kept) <= set(inner_planted)
