@@ -27,6 +27,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+import dynamic_block_sparse_proxy_b200 as crisp  # noqa: E402  (the library loads on first use)
 from dynamic_block_sparse_proxy_b200 import workloads as W  # noqa: E402
 
 METRIC = "prefill tokens/s per layer (select+sparse attn) at 128k; % bf16 peak, % HBM BW"
@@ -117,8 +118,8 @@ def select_bytes(w, n_pe_heads: int, total_pairs: int) -> float:
 # workload, from a one-pass ncu capture of this command's own launch. The figure belongs to the
 # kernel source it was taken on; for any other source or workload the bench reports null.
 ATTN_TRAFFIC = {"workload": "llama8b_128k",
-                "source_sha256": "dbf0c5bc3904b8f90c36365e07edbb601bf513b9e713c7b5a2334e35ade98f59",
-                "bytes": 2.73e9 + 1.06e9}
+                "source_sha256": "7054caa5815700d80cac3ad12fe8f9f681f6e55e29d62e7fb58b6b6c14a9577f",
+                "bytes": 2.69e9 + 1.06e9}
 
 
 def attn_traffic(w):
@@ -130,14 +131,48 @@ def attn_traffic(w):
     return ATTN_TRAFFIC["bytes"]
 
 
+# Index-selection rules: CRISP's own (default), the FlexPrefill baseline the CRISP paper compares
+# against, and CRISP's variants (median floor, the speed-focused alpha values).
+RULES = {
+    "crisp": crisp.Params(),
+    "flexprefill": crisp.Params.flexprefill(),
+    "crisp_median": crisp.Params(floor_rule=1),
+    "crisp_alpha1.25": crisp.Params(alpha=1.25),
+    "crisp_alpha1.5": crisp.Params(alpha=1.5),
+}
+
+
+def rule_config(p) -> dict:
+    out = {"tau_proxy": p.tau_proxy, "alpha": p.alpha, "gamma": p.gamma, "min_blocks": p.min_blocks}
+    if p.route_rule:
+        out.update(route="jsd", tau_jsd=p.tau_jsd)
+    if p.vs_rule:
+        out["vs"] = "gamma per direction"
+    if p.floor_rule:
+        out["floor"] = "median"
+    return out
+
+
+def bench_config(w, args, world: int) -> dict:
+    """The workload line both arms (CUDA and oracle) report."""
+    return {"workload": w.name, "n": w.n, "h_q": w.h_q, "h_kv": w.h_kv, "d": w.d, "block": 128,
+            "rules": args.rules, **rule_config(RULES[args.rules]),
+            "parallelism": f"independent layer per rank x{world}",
+            "l2": "flushed before every step (256 MB write); inputs also exceed L2"}
+
+
+def oracle_kwargs(p) -> dict:
+    return dict(tau_proxy=p.tau_proxy, alpha=p.alpha, gamma=p.gamma, min_blocks=p.min_blocks,
+                route_rule="jsd" if p.route_rule else "cstruct", tau_jsd=p.tau_jsd,
+                vs_rule="gamma" if p.vs_rule else "floor", floor="median" if p.floor_rule else "mean")
+
+
 def attn_flops(total_pairs: int, d: int = 128) -> float:
     return W.block_pair_flops(d) * total_pairs
 
 
 # ---------------------------------------------------------------------------- GPU arm
 def run_crisp(args):
-    import dynamic_block_sparse_proxy_b200 as crisp
-
     world, rank, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -150,7 +185,7 @@ def run_crisp(args):
     if args.n:
         w = w.scaled(args.n)
     q, k, v, meta = W.generate(w, device=dev)
-    params = crisp.Params()
+    params = RULES[args.rules]
     ws = crisp.workspace(w.h_q, w.h_kv, w.n, dev)
     idx = crisp.Index.empty(w.h_q, w.n, dev)
     o = torch.empty_like(q)
@@ -255,10 +290,7 @@ def run_crisp(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded planted-structure generator)",
-        "config": {"workload": w.name, "n": w.n, "h_q": w.h_q, "h_kv": w.h_kv, "d": w.d,
-                   "block": 128, "tau_proxy": 0.5, "alpha": 1.0, "gamma": 0.95, "min_blocks": 0,
-                   "parallelism": f"independent layer per rank x{world}",
-                   "l2": "flushed before every step (256 MB write); inputs also exceed L2"},
+        "config": bench_config(w, args, world),
         "roofline": {"bound": "tensor", "kernel": "sparse_attn", "achieved": achieved_tf,
                      "peak": sustained, "unit": "TFLOP/s", "frac": achieved_tf / sustained,
                      "peak_kind": f"bf16 sustained ({src})",
@@ -275,14 +307,14 @@ def run_crisp(args):
         "clocks": clocks,
     }
     if args.cpu_baseline:
-        out["cpu_baseline"] = oracle_baseline(w, q, k, v, idx, args.cpu_seconds)
+        out["cpu_baseline"] = oracle_baseline(w, q, k, v, idx, args.cpu_seconds, params=params)
     print(json.dumps(out), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
 
 
 # ---------------------------------------------------------------------------- CPU oracle arm
-def oracle_baseline(w, q, k, v, idx, budget_s: float, seed: int = 0) -> dict:
+def oracle_baseline(w, q, k, v, idx, budget_s: float, seed: int = 0, params=None) -> dict:
     """Time the fp64 oracle on a bounded sample of the workload and extrapolate to one layer:
     selection of one Vertical-Slash and one Pooled-Estimation head (scaled by the head counts),
     and attention on a sample of query blocks (scaled by selected block pairs)."""
@@ -301,7 +333,7 @@ def oracle_baseline(w, q, k, v, idx, budget_s: float, seed: int = 0) -> dict:
     for h in heads:
         qh, kh = f64(q[h]), f64(k[h // G])
         t0 = time.perf_counter()
-        sel[h] = O.select_head(qh, kh)
+        sel[h] = O.select_head(qh, kh, **oracle_kwargs(params or crisp.Params()))
         times[h] = time.perf_counter() - t0
     n_vs = int(route.sum()) if route is not None else sum(conc)
     n_pe = w.h_q - n_vs
@@ -345,13 +377,16 @@ def run_reference(args):
     if rank != 0:
         return
     w = W.WORKLOADS[args.workload]
+    if args.n:
+        w = w.scaled(args.n)
     torch.manual_seed(0)
     q, k, v, meta = W.generate(w, device="cuda" if torch.cuda.is_available() else "cpu")
     vals = []
     t0 = time.perf_counter()
     base = None
     for i in range(args.warmup + args.steps):
-        b = oracle_baseline(w, q, k, v, None, args.cpu_seconds / max(1, args.steps + args.warmup), seed=i)
+        b = oracle_baseline(w, q, k, v, None, args.cpu_seconds / max(1, args.steps + args.warmup), seed=i,
+                            params=RULES[args.rules])
         if i >= args.warmup:
             vals.append(b["value"])
             base = b
@@ -359,7 +394,7 @@ def run_reference(args):
     out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": w.n / value * 1e3, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": {"workload": w.name, "n": w.n, "h_q": w.h_q, "h_kv": w.h_kv, "d": w.d},
+           "config": bench_config(w, args, world),
            "impl": "reference",
            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": base["cores"], "kind": "oracle",
                             "sample": base["sample"]},
@@ -375,6 +410,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="crisp", choices=["crisp", "reference"])
+    ap.add_argument("--rules", default="crisp", choices=sorted(RULES),
+                    help="index-selection rules (the headline metric uses CRISP's own)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")

@@ -34,7 +34,9 @@ class CrispError(RuntimeError):
 
 class _Params(ctypes.Structure):
     _fields_ = [("block", ctypes.c_int32), ("anchors", ctypes.c_int32), ("tau_proxy", ctypes.c_float),
-                ("alpha", ctypes.c_float), ("gamma", ctypes.c_float), ("min_blocks", ctypes.c_int32)]
+                ("alpha", ctypes.c_float), ("gamma", ctypes.c_float), ("min_blocks", ctypes.c_int32),
+                ("route_rule", ctypes.c_int32), ("tau_jsd", ctypes.c_float), ("vs_rule", ctypes.c_int32),
+                ("floor_rule", ctypes.c_int32)]
 
 
 class _Index(ctypes.Structure):
@@ -73,16 +75,29 @@ def lib() -> ctypes.CDLL:
 
 @dataclasses.dataclass
 class Params:
-    """CRISP parameters (paper §3.2, §4, §5). block and anchors must be 128."""
+    """CRISP parameters (paper §3.2, §4, §5). block and anchors must be 128.
+
+    route_rule / vs_rule / floor_rule select the FlexPrefill baseline rules (JSD router,
+    per-direction gamma cut) and the median noise floor; 0 is CRISP's own rule."""
     block: int = 128
     anchors: int = 128
     tau_proxy: float = 0.5
     alpha: float = 1.0
     gamma: float = 0.95
     min_blocks: int = 0
+    route_rule: int = 0
+    tau_jsd: float = 0.1
+    vs_rule: int = 0
+    floor_rule: int = 0
+
+    @staticmethod
+    def flexprefill(**kw) -> "Params":
+        """FlexPrefill's rules as the CRISP paper describes them (JSD router, gamma per direction)."""
+        return Params(route_rule=1, vs_rule=1, **kw)
 
     def c(self) -> _Params:
-        return _Params(self.block, self.anchors, self.tau_proxy, self.alpha, self.gamma, self.min_blocks)
+        return _Params(self.block, self.anchors, self.tau_proxy, self.alpha, self.gamma, self.min_blocks,
+                       self.route_rule, self.tau_jsd, self.vs_rule, self.floor_rule)
 
 
 @dataclasses.dataclass
@@ -92,7 +107,7 @@ class Index:
     c_struct: torch.Tensor   # float32 [h_q]
     row_ptr: torch.Tensor    # int32 [h_q, N_b+1]
     cols: torch.Tensor       # int32 [h_q, N_b(N_b+1)/2]
-    debug: torch.Tensor | None = None  # float32 [h_q, 2*N_b+4]
+    debug: torch.Tensor | None = None  # float32 [h_q, 2*N_b+5]
 
     @staticmethod
     def empty(h_q: int, n: int, device, debug: bool = False) -> "Index":
@@ -100,7 +115,7 @@ class Index:
         i32 = dict(device=device, dtype=torch.int32)
         return Index(torch.empty(h_q, **i32), torch.empty(h_q, device=device, dtype=torch.float32),
                      torch.empty(h_q, nb + 1, **i32), torch.empty(h_q, nb * (nb + 1) // 2, **i32),
-                     torch.empty(h_q, 2 * nb + 4, device=device, dtype=torch.float32) if debug else None)
+                     torch.empty(h_q, 2 * nb + 5, device=device, dtype=torch.float32) if debug else None)
 
     def c(self) -> _Index:
         return _Index(self.route.data_ptr(), self.c_struct.data_ptr(), self.row_ptr.data_ptr(),

@@ -64,6 +64,9 @@ int check_params(const crisp_params* p) {
   if (!std::isfinite(p->tau_proxy) || !std::isfinite(p->alpha) || !std::isfinite(p->gamma))
     return CRISP_ERR_INVALID_ARG;
   if (p->alpha < 0.f || p->gamma <= 0.f || p->min_blocks < 0) return CRISP_ERR_INVALID_ARG;
+  if ((p->route_rule != 0 && p->route_rule != 1) || (p->vs_rule != 0 && p->vs_rule != 1) ||
+      (p->floor_rule != 0 && p->floor_rule != 1) || !std::isfinite(p->tau_jsd) || p->tau_jsd < 0.f)
+    return CRISP_ERR_INVALID_ARG;
   return CRISP_OK;
 }
 
@@ -94,6 +97,10 @@ int run_select(const void* q, const void* k, const Shape& s, const crisp_params*
   a.alpha = p->alpha;
   a.gamma = p->gamma;
   a.min_blocks = p->min_blocks;
+  a.route_rule = p->route_rule;
+  a.tau_jsd = p->tau_jsd;
+  a.vs_rule = p->vs_rule;
+  a.floor_rule = p->floor_rule;
   a.status = at<int>(ws, w.status);
   a.trace = at<unsigned long long>(ws, w.trace);
   a.part = at<float2>(ws, w.part);
@@ -200,6 +207,7 @@ int crisp_select(const void* q, const void* k, int h_q, int h_kv, int n, int d, 
   Shape s;
   int rc = check_shape(h_q, h_kv, n, d, &s);
   if (rc == CRISP_OK) rc = check_params(params);
+  if (rc == CRISP_OK && s.nb > kMaxSelectBlocks) rc = CRISP_ERR_UNSUPPORTED;
   if (rc == CRISP_OK && !tensors_ok(q, k, nullptr)) rc = CRISP_ERR_INVALID_ARG;
   if (rc == CRISP_OK) rc = check_index(out, true);
   if (rc == CRISP_OK) rc = check_ws(ws, ws_bytes, s);
@@ -226,6 +234,7 @@ int crisp_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv
   Shape s;
   int rc = check_shape(h_q, h_kv, n, d, &s);
   if (rc == CRISP_OK) rc = check_params(params);
+  if (rc == CRISP_OK && s.nb > kMaxSelectBlocks) rc = CRISP_ERR_UNSUPPORTED;
   if (rc == CRISP_OK && (!tensors_ok(q, k, v) || v == nullptr || o == nullptr || !aligned(o, 16)))
     rc = CRISP_ERR_INVALID_ARG;
   if (rc == CRISP_OK && idx_out != nullptr) rc = check_index(idx_out, true);

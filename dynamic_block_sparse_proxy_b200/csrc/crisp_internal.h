@@ -15,7 +15,8 @@ namespace crisp {
 constexpr int kB = 128;        // block size (queries and keys)
 constexpr int kD = 128;        // head dimension
 constexpr int kProxyChunk = 16;  // key blocks per proxy CTA
-constexpr int kHistBins = 2048;  // radix-select bins per pass (11, 10, 10 bits)
+constexpr int kHistBins = 2048;
+constexpr int kMaxSelectBlocks = 8192;  // selection keeps per-head block arrays in shared memory  // radix-select bins per pass (11, 10, 10 bits)
 constexpr double kMassUnit = 1099511627776.0;  // 2^40: fixed-point scale of histogram masses
 
 struct Shape {
@@ -84,6 +85,10 @@ struct SelectArgs {
   Shape s;
   float tau, alpha, gamma;
   int min_blocks;
+  int route_rule;  // 0: C_struct >= tau; 1: JSD(a_bar, a_hat) >= tau_jsd
+  float tau_jsd;
+  int vs_rule;     // 0: noise-floor keep rule; 1: per-direction gamma cut
+  int floor_rule;  // 0: mean floor; 1: median floor
   int* status;
   unsigned long long* trace;
   float2* part;

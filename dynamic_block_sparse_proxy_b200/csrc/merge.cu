@@ -217,7 +217,7 @@ __global__ void __launch_bounds__(1024) scan_rows_kernel(const int* in, int* out
   }
   if (threadIdx.x == 0) {
     dst[nb] = (int)carry;
-    if (debug_total != nullptr) debug_total[(size_t)h * (2 * nb + 4) + 2 * nb + 3] = (float)carry;
+    if (debug_total != nullptr) debug_total[(size_t)h * (2 * nb + 5) + 2 * nb + 3] = (float)carry;
   }
 }
 

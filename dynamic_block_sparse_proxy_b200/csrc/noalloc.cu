@@ -84,6 +84,10 @@ extern "C" int crisp_select_noalloc(const void* q, const void* k, int h_q, int h
   const long long nb = n / kB;
   const long long cap = nb * (nb + 1) / 2;
   if (cap > 0x7fffffffLL || (long long)h_q * n > 0x7fffffffLL) return CRISP_ERR_OVERFLOW;
+  if (nb > kMaxSelectBlocks) return CRISP_ERR_UNSUPPORTED;
+  if ((p->route_rule != 0 && p->route_rule != 1) || (p->vs_rule != 0 && p->vs_rule != 1) ||
+      (p->floor_rule != 0 && p->floor_rule != 1) || !std::isfinite(p->tau_jsd) || p->tau_jsd < 0.f)
+    return CRISP_ERR_INVALID_ARG;
   Shape s;
   s.h_q = h_q;
   s.h_kv = h_kv;
@@ -107,6 +111,10 @@ extern "C" int crisp_select_noalloc(const void* q, const void* k, int h_q, int h
   a.alpha = p->alpha;
   a.gamma = p->gamma;
   a.min_blocks = p->min_blocks;
+  a.route_rule = p->route_rule;
+  a.tau_jsd = p->tau_jsd;
+  a.vs_rule = p->vs_rule;
+  a.floor_rule = p->floor_rule;
   a.status = device_status != nullptr ? device_status : reinterpret_cast<int*>(at(w.status));
   a.trace = reinterpret_cast<unsigned long long*>(at(w.trace));
   a.part = reinterpret_cast<float2*>(at(w.part));

@@ -8,12 +8,15 @@
 //   2. p_v[kb] = sum_r w*(lo+hi) (vertical block mass), and the slash block masses
 //      p_s[N_b-1-kb] += sum_r w*lo, p_s[N_b-2-kb] += sum_r w*hi (CRISP §4, both directions);
 //   3. C_struct = p_v[0] + p_v[N_b-1], the mass on the first and last 128 keys (CRISP §3.2);
-//      route = Vertical-Slash iff C_struct >= tau_proxy;
+//      route = Vertical-Slash iff C_struct >= tau_proxy (or, with the FlexPrefill router the
+//      CRISP paper compares against, iff JSD(a_bar, a_hat) >= tau_jsd);
 //   4. per direction the noise floor mu = (mass of blocks 1..N_b-2) / (N_b-2). The block masses
 //      add up to one, so this is max(1 - p[0] - p[N_b-1], 0) / (N_b-2) of CRISP §4 summed
 //      without the cancellation that subtracting a near-one sink mass from 1 would cause;
 //   5. keep block j in [1, N_b-2] iff p[j] > alpha*mu (strict), then top up to min_blocks with
-//      the largest remaining blocks (ties to the lower index).
+//      the largest remaining blocks (ties to the lower index). Variants: mu as the median of
+//      p[1..N_b-2]; or FlexPrefill's per-direction cut, the shortest (p desc, index asc) prefix
+//      reaching gamma of the direction's mass.
 // Reductions run in fp64.
 #include "crisp_internal.h"
 #include "sm100.cuh"
@@ -118,16 +121,177 @@ __global__ void __launch_bounds__(MASS_WARPS * 32) block_mass_kernel(const Selec
   }
 }
 
-// 3. Per head: C_struct, route, noise floors, keep flags (+ top-up).
+// Block-wide maximum and sum of doubles (all threads receive the result).
+__device__ double block_max(double v, double* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  double t = -INFINITY;
+  for (int i = 0; i < NWARP; ++i) t = fmax(t, red[i]);
+  return t;
+}
+
+// FlexPrefill's routing statistic (route_rule 1): JSD between a_bar, the softmax over all key
+// blocks of the last query block's mean query against the key-block means (1/sqrt(d) scale),
+// and a_hat, the proxy's per-query mean pooled to blocks (p_v, normalised to sum 1). Natural
+// logarithm, 0 log 0 = 0. `abar` is scratch for N_b doubles; `qpart` stages the query mean.
+__device__ double jsd_statistic(const SelectArgs& a, int h, const double* pv, double* abar, float* qm,
+                                float (*qpart)[kD], double* red) {
+  const Shape& s = a.s;
+  const int nb = s.nb, tid = threadIdx.x, kv = h / s.G;
+  // mean of the last 128 query rows; thread t sums column t%128 over rows t/128, t/128+4, ...
+  {
+    const int col = tid & (kD - 1), rg = tid >> 7;
+    const __nv_bfloat16* qrow = a.q + ((size_t)h * s.n + (size_t)(s.n - kB)) * kD + col;
+    float acc = 0.f;
+    for (int r = rg; r < kB; r += THREADS / kD) acc += __bfloat162float(qrow[(size_t)r * kD]);
+    qpart[rg][col] = acc;
+    __syncthreads();
+    if (tid < kD) {
+      float t = 0.f;
+      for (int g = 0; g < THREADS / kD; ++g) t += qpart[g][tid];
+      qm[tid] = t * (1.f / kB);
+    }
+    __syncthreads();
+  }
+  // logits and softmax over the key blocks
+  const double inv_sqrt_d = 0.08838834764831845;
+  double mx = -INFINITY;
+  for (int kb = tid; kb < nb; kb += THREADS) {
+    const float4* kr = reinterpret_cast<const float4*>(a.kbar + ((size_t)kv * nb + kb) * kD);
+    double dot = 0.0;
+#pragma unroll 4
+    for (int i = 0; i < kD / 4; ++i) {
+      const float4 kk = kr[i];
+      dot += (double)qm[4 * i] * kk.x + (double)qm[4 * i + 1] * kk.y + (double)qm[4 * i + 2] * kk.z +
+             (double)qm[4 * i + 3] * kk.w;
+    }
+    abar[kb] = dot * inv_sqrt_d;
+    mx = fmax(mx, abar[kb]);
+  }
+  mx = block_max(mx, red);
+  double z = 0.0, spv = 0.0;
+  for (int kb = tid; kb < nb; kb += THREADS) {
+    abar[kb] = exp(abar[kb] - mx);
+    z += abar[kb];
+    spv += pv[kb];
+  }
+  z = block_sum(z, red);
+  spv = block_sum(spv, red);
+  double t = 0.0;
+  for (int kb = tid; kb < nb; kb += THREADS) {
+    const double p = abar[kb] / z, q = pv[kb] / spv, m = 0.5 * (p + q);
+    if (p > 0.0) t += p * log(p / m);
+    if (q > 0.0) t += q * log(q / m);
+  }
+  return 0.5 * block_sum(t, red);
+}
+
+// Sorts the indices 0..P2-1 in sidx so that (p desc, index asc) order holds for the indices
+// `member` accepts; all others go last. P2 is a power of two >= the number of indices.
+template <typename Member>
+__device__ void sort_desc(const double* p, int* sidx, int P2, Member member) {
+  for (int i = threadIdx.x; i < P2; i += THREADS) sidx[i] = i;
+  __syncthreads();
+  auto before = [&](int x, int y) {  // x strictly before y
+    const bool mx = member(x), my = member(y);
+    if (mx != my) return mx;
+    if (!mx) return x < y;
+    return p[x] > p[y] || (p[x] == p[y] && x < y);
+  };
+  for (int k = 2; k <= P2; k <<= 1)
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < P2; i += THREADS) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const int x = sidx[i], y = sidx[ixj];
+          const bool asc = (i & k) == 0;  // this pair's sequence runs in the final order
+          if (asc ? before(y, x) : before(x, y)) {
+            sidx[i] = y;
+            sidx[ixj] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+}
+
+// FlexPrefill's per-direction cut (vs_rule 1): the shortest prefix of the blocks sorted
+// (p desc, index asc) whose sum reaches gamma * sum(p); sets flags on its blocks in
+// [1, N_b-2] and returns the value of the last block kept.
+__device__ double gamma_direction(const double* p, int* sidx, int nb, int P2, double gamma, uint8_t* flags,
+                                  double* red, int* pos_min) {
+  sort_desc(p, sidx, P2, [nb](int x) { return x < nb; });
+  double tot = 0.0;
+  for (int i = threadIdx.x; i < nb; i += THREADS) tot += p[i];
+  tot = block_sum(tot, red);
+  const double target = gamma * tot;
+  // per-thread contiguous segment of the sorted order, then a block exclusive scan of segments
+  const int seg = (nb + THREADS - 1) / THREADS;
+  const int b0 = threadIdx.x * seg, b1 = min(nb, b0 + seg);
+  double local = 0.0;
+  for (int i = b0; i < b1; ++i) local += p[sidx[i]];
+  // exclusive scan over threads (warp shuffles, then warp totals)
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  double incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  __syncthreads();
+  if (lane == 31) red[w] = incl;
+  if (threadIdx.x == 0) *pos_min = nb;
+  __syncthreads();
+  double base = incl - local;
+  for (int i = 0; i < w; ++i) base += red[i];
+  double c = base;
+  for (int i = b0; i < b1; ++i) {
+    c += p[sidx[i]];
+    if (c >= target) {
+      atomicMin(pos_min, i);
+      break;
+    }
+  }
+  __syncthreads();
+  const int count = min(*pos_min + 1, nb);
+  for (int i = threadIdx.x; i < nb; i += THREADS) {
+    const int j = sidx[i];
+    if (j >= 1 && j <= nb - 2) flags[j] = i < count ? 1 : 0;
+  }
+  const double cut = p[sidx[count - 1]];
+  __syncthreads();
+  return cut;
+}
+
+// The median of p[1..N_b-2] (mean of the two middle values for an even count).
+__device__ double median_inner(const double* p, int* sidx, int nb, int P2) {
+  sort_desc(p, sidx, P2, [nb](int x) { return x >= 1 && x <= nb - 2; });
+  const int m = nb - 2;
+  const double lo = p[sidx[(m - 1) / 2]], hi = p[sidx[m / 2]];
+  const double med = 0.5 * (lo + hi);
+  __syncthreads();
+  return med;
+}
+
+// 3. Per head: C_struct (or the JSD), route, noise floors, keep flags (+ top-up).
 __global__ void __launch_bounds__(THREADS) route_threshold_kernel(const SelectArgs a) {
   extern __shared__ double dsm[];
   const Shape& s = a.s;
   const int nb = s.nb, h = blockIdx.x, tid = threadIdx.x;
-  double* pv = dsm;       // [nb]
-  double* ps = dsm + nb;  // [nb]
+  double* pv = dsm;        // [nb]
+  double* ps = dsm + nb;   // [nb]
+  double* aux = dsm + 2 * nb;                  // [nb] doubles: a_bar, then sort indices
+  int* sidx = reinterpret_cast<int*>(aux);     // [P2] ints (P2 <= 2 nb)
   __shared__ double red[NWARP];
   __shared__ double redv[NWARP];
   __shared__ int redi[NWARP];
+  __shared__ float qm[kD];
+  __shared__ float qpart[THREADS / kD][kD];
+  __shared__ int pos_min;
   for (int i = tid; i < nb; i += THREADS) {
     pv[i] = a.pv[(size_t)h * nb + i];
     ps[i] = a.ps_lo[(size_t)h * nb + i] + (i == nb - 1 ? 0.0 : a.ps_hi[(size_t)h * nb + i]);
@@ -136,44 +300,59 @@ __global__ void __launch_bounds__(THREADS) route_threshold_kernel(const SelectAr
 
   // C_struct and route
   const double C = nb >= 2 ? pv[0] + pv[nb - 1] : pv[0];
-  const int vs = C >= (double)a.tau ? 1 : 0;
-
-  // noise floors
-  double mu_v = 0.0, mu_s = 0.0;
-  if (nb >= 3) {
-    double rv = 0.0, rs = 0.0;
-    for (int j = 1 + tid; j <= nb - 2; j += THREADS) {
-      rv += pv[j];
-      rs += ps[j];
-    }
-    rv = block_sum(rv, red);
-    rs = block_sum(rs, red);
-    mu_v = rv / (nb - 2);
-    mu_s = rs / (nb - 2);
+  double jsd = 0.0;
+  int vs;
+  if (a.route_rule == 1) {
+    jsd = jsd_statistic(a, h, pv, aux, qm, qpart, red);
+    vs = jsd >= (double)a.tau_jsd ? 1 : 0;
+  } else {
+    vs = C >= (double)a.tau ? 1 : 0;
   }
+  __syncthreads();
 
-  // keep flags (+ top-up)
+  // keep flags per direction
   uint8_t* kv_out = a.keep_v + (size_t)h * nb;
   uint8_t* ks_out = a.keep_s + (size_t)h * nb;
   const double alpha = (double)a.alpha;
-  int nv = 0, ns = 0;
-  for (int j = tid; j < nb; j += THREADS) {
-    const bool inner = nb >= 3 && j >= 1 && j <= nb - 2;
-    const uint8_t fv = inner && pv[j] > alpha * mu_v;
-    const uint8_t fs = inner && ps[j] > alpha * mu_s;
-    kv_out[j] = fv;
-    ks_out[j] = fs;
-    nv += fv;
-    ns += fs;
+  int P2 = 1;
+  while (P2 < nb) P2 <<= 1;
+  double mu_out[2] = {0.0, 0.0};
+  int nkeep[2] = {0, 0};
+  for (int dir = 0; dir < 2; ++dir) {
+    const double* p = dir == 0 ? pv : ps;
+    uint8_t* flags = dir == 0 ? kv_out : ks_out;
+    for (int j = tid; j < nb; j += THREADS) flags[j] = 0;
+    __syncthreads();
+    if (nb >= 3) {
+      if (a.vs_rule == 1) {
+        if (vs) mu_out[dir] = gamma_direction(p, sidx, nb, P2, (double)a.gamma, flags, red, &pos_min);
+      } else {
+        double mu;
+        if (a.floor_rule == 1) {
+          mu = median_inner(p, sidx, nb, P2);
+        } else {
+          // mean residual mass of blocks 1..N_b-2: their sum, without subtracting from 1
+          double r = 0.0;
+          for (int j = 1 + tid; j <= nb - 2; j += THREADS) r += p[j];
+          mu = block_sum(r, red) / (nb - 2);
+        }
+        mu_out[dir] = mu;
+        for (int j = 1 + tid; j <= nb - 2; j += THREADS) flags[j] = p[j] > alpha * mu ? 1 : 0;
+      }
+    }
+    __syncthreads();
+    int cnt = 0;
+    for (int j = tid; j < nb; j += THREADS) cnt += flags[j];
+    nkeep[dir] = (int)block_sum((double)cnt, red);
   }
-  nv = (int)block_sum((double)nv, red);
-  ns = (int)block_sum((double)ns, red);
+
+  // top-up to min_blocks (both rules)
   if (vs && nb >= 3 && a.min_blocks > 0) {
     __syncthreads();
     for (int dir = 0; dir < 2; ++dir) {
       uint8_t* flags = dir == 0 ? kv_out : ks_out;
       const double* p = dir == 0 ? pv : ps;
-      int have = dir == 0 ? nv : ns;
+      int have = nkeep[dir];
       const int want = min(a.min_blocks, nb - 2);
       while (have < want) {
         double bv = 0.0;
@@ -198,15 +377,16 @@ __global__ void __launch_bounds__(THREADS) route_threshold_kernel(const SelectAr
     a.c_struct[h] = (float)C;
   }
   if (a.debug != nullptr) {
-    float* dbg = a.debug + (size_t)h * (2 * nb + 4);
+    float* dbg = a.debug + (size_t)h * (2 * nb + 5);
     for (int j = tid; j < nb; j += THREADS) {
       dbg[j] = (float)pv[j];
       dbg[nb + j] = (float)ps[j];
     }
     if (tid == 0) {
-      dbg[2 * nb] = (float)mu_v;
-      dbg[2 * nb + 1] = (float)mu_s;
+      dbg[2 * nb] = (float)mu_out[0];
+      dbg[2 * nb + 1] = (float)mu_out[1];
       dbg[2 * nb + 2] = (float)C;
+      dbg[2 * nb + 4] = (float)jsd;
     }
   }
 }
@@ -216,7 +396,7 @@ __global__ void __launch_bounds__(THREADS) route_threshold_kernel(const SelectAr
 cudaError_t launch_route_threshold(const SelectArgs& a, cudaStream_t st) {
   row_stats_kernel<<<dim3(kB / STAT_ROWS, a.s.h_q), STAT_ROWS * 32, 0, st>>>(a);
   block_mass_kernel<<<dim3((a.s.nb + MASS_WARPS - 1) / MASS_WARPS, a.s.h_q), MASS_WARPS * 32, 0, st>>>(a);
-  const size_t smem = (size_t)2 * a.s.nb * sizeof(double);
+  const size_t smem = (size_t)3 * a.s.nb * sizeof(double);  // p_v, p_s, and a_bar / sort indices
   cudaError_t e = cudaFuncSetAttribute(route_threshold_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

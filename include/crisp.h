@@ -57,6 +57,22 @@ enum {
  *   gamma      Pooled-Estimation coverage target of the global cumulative cut (gamma > 0;
  *              gamma >= 1 keeps every causal block)
  *   min_blocks minimum kept blocks per direction on Vertical-Slash heads (>= 0; 0 = off)
+ * Rule switches (0 = CRISP, the default for a zero-initialised field):
+ *   route_rule 0: C_struct >= tau_proxy. 1: FlexPrefill's router as the CRISP paper describes
+ *              it (§2): VS iff JSD(a_bar, a_hat) >= tau_jsd, a_bar the softmax over key blocks of
+ *              the last query block's mean query against the key-block means (1/sqrt(d) scale),
+ *              a_hat the proxy's per-query mean pooled to blocks (p_v); natural logarithm.
+ *   tau_jsd    threshold of route_rule 1 (finite, >= 0)
+ *   vs_rule    0: the noise-floor keep rule above. 1: FlexPrefill's per-direction cut (§2):
+ *              each direction keeps the shortest prefix of its blocks sorted (p desc, index asc)
+ *              whose sum reaches gamma times the direction's total (first and last blocks are
+ *              kept either way; min_blocks still tops up)
+ *   floor_rule 0: mu is the mean residual mass above. 1: mu is the median of p[1..N_b-2] (the
+ *              median floor of the paper's robustness discussion, §4 / Table 9)
+ * Selection (crisp_select, crisp_prefill, crisp_select_noalloc) keeps per-head block arrays in
+ * shared memory and supports N_b <= 8192 (n <= 1,048,576); larger n returns
+ * CRISP_ERR_UNSUPPORTED. Attention alone (crisp_sparse_prefill, crisp_dense_prefill) has no
+ * such limit.
  */
 typedef struct {
   int32_t block;
@@ -65,6 +81,10 @@ typedef struct {
   float alpha;
   float gamma;
   int32_t min_blocks;
+  int32_t route_rule;
+  float tau_jsd;
+  int32_t vs_rule;
+  int32_t floor_rule;
 } crisp_params;
 
 /*
@@ -75,8 +95,10 @@ typedef struct {
  *   row_ptr  int32 [h_q][N_b+1] row qb of head h spans cols[h*cap + row_ptr[h][qb] ..
  *                               h*cap + row_ptr[h][qb+1]), cap = N_b*(N_b+1)/2
  *   cols     int32 [h_q][cap]   key-block indices, strictly ascending within a row, each <= qb
- *   debug    float [h_q][2*N_b+4] or NULL: p_v[N_b], p_s[N_b] (vertical and slash block
- *            masses, CRISP §4), then mu_v, mu_s, C_struct, and the number of selected pairs
+ *   debug    float [h_q][2*N_b+5] or NULL: p_v[N_b], p_s[N_b] (vertical and slash block
+ *            masses, CRISP §4), then mu_v, mu_s, C_struct, the number of selected pairs, and
+ *            the JSD of route_rule 1 (0 otherwise). With vs_rule 1, mu_v and mu_s hold the value
+ *            of the last block each direction's cut kept.
  */
 typedef struct {
   int32_t* route;

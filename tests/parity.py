@@ -18,6 +18,7 @@ ATTN_MAX_ABS = 2e-2
 ATTN_MEAN_ABS = 2e-3
 LSE_ABS = 5e-3
 P_REL = 2e-4     # relative agreement of the block masses p_v, p_s (fp32 path vs fp64)
+JSD_REL = 2e-4   # JSD: a_bar comes from fp32 pooled means, a_hat from the fp32 proxy
 
 
 def f32(x: float) -> float:
@@ -27,7 +28,9 @@ def f32(x: float) -> float:
 
 def oracle_params(params) -> dict:
     return dict(block=params.block, anchors=params.anchors, tau_proxy=f32(params.tau_proxy),
-                alpha=f32(params.alpha), gamma=f32(params.gamma), min_blocks=params.min_blocks)
+                alpha=f32(params.alpha), gamma=f32(params.gamma), min_blocks=params.min_blocks,
+                route_rule="jsd" if params.route_rule else "cstruct", tau_jsd=f32(params.tau_jsd),
+                vs_rule="gamma" if params.vs_rule else "floor", floor="median" if params.floor_rule else "mean")
 
 
 def f64(t: torch.Tensor) -> np.ndarray:
@@ -56,10 +59,12 @@ def compare_selection(index, sels: dict, nb: int, log: list | None = None) -> di
     for h, s in sels.items():
         stats["heads"] += 1
         assert abs(float(cst[h]) - s["c_struct"]) <= 1e-5 * max(1.0, s["c_struct"]) + 1e-6, (h, cst[h], s["c_struct"])
+        if dbg is not None and "jsd" in s:
+            assert abs(float(dbg[h, 2 * nb + 4]) - s["jsd"]) <= JSD_REL * max(s["jsd"], 1e-3), (h, dbg[h, 2 * nb + 4], s["jsd"])
         if s["route_tie"]:
             stats["route_ties"] += 1
             if log is not None:
-                log.append(f"head {h}: C_struct {s['c_struct']:.8f} within the tie band of tau")
+                log.append(f"head {h}: routing statistic within the tie band of its threshold")
             continue
         assert int(route[h]) == s["route"], (h, route[h], s["route"], s["c_struct"])
         if dbg is not None:

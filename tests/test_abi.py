@@ -80,10 +80,22 @@ def test_select_rejects_bad_arguments_before_launch(L):
     for args, want in cases:
         assert crisp.STATUS_NAMES[L.crisp_select(*args)] == want, args
     for bad in (crisp.Params(alpha=-1.0), crisp.Params(gamma=0.0), crisp.Params(min_blocks=-1),
-                crisp.Params(tau_proxy=float("nan")), crisp.Params(anchors=64)):
+                crisp.Params(tau_proxy=float("nan")), crisp.Params(anchors=64), crisp.Params(route_rule=2),
+                crisp.Params(vs_rule=-1), crisp.Params(floor_rule=3), crisp.Params(tau_jsd=-0.5),
+                crisp.Params(tau_jsd=float("inf"))):
         bp = bad.c()
         rc = L.crisp_select(fake, fake, 1, 1, 4096, 128, ctypes.byref(bp), ctypes.byref(ix), ws, big, None)
         assert rc in (-1, -2), bad
+
+
+def test_selection_beyond_8192_blocks_is_unsupported(L):
+    p = crisp.Params().c()
+    ix = _idx()
+    n = 128 * 8193
+    rc = L.crisp_select(0x10000, 0x10000, 1, 1, n, 128, ctypes.byref(p), ctypes.byref(ix), 0x100000, 1 << 40, None)
+    assert rc == -2
+    rc = L.crisp_select_noalloc(0x10000, 0x10000, 1, 1, n, 128, ctypes.byref(p), ctypes.byref(ix), None, None)
+    assert rc == -2
 
 
 def test_attention_entry_points_reject_bad_arguments(L):

@@ -262,6 +262,62 @@ def test_bad_arguments_raise():
     assert crisp.get_status(ws) == 0
 
 
+# ------------------------------------------------------------- FlexPrefill rules, median floor, alpha
+RULES = {
+    "flexprefill": crisp.Params.flexprefill(),
+    "jsd_route_only": crisp.Params(route_rule=1),
+    "gamma_vs_only": crisp.Params(vs_rule=1),
+    "median_floor": crisp.Params(floor_rule=1),
+    "median_floor_min8": crisp.Params(floor_rule=1, min_blocks=8),
+    "alpha_1.25": crisp.Params(alpha=1.25),
+    "alpha_1.5": crisp.Params(alpha=1.5),
+    "flexprefill_gamma_0.9": crisp.Params.flexprefill(gamma=0.9),
+}
+
+
+@pytest.mark.parametrize("rule", sorted(RULES))
+@pytest.mark.parametrize("name,n", [("llama8b_32k", 8192), ("qwen7b_128k", 4096)])
+def test_rule_variants_match_oracle(rule, name, n):
+    params = RULES[rule]
+    w = W.WORKLOADS[name].scaled(n)
+    q, k, v, meta = W.generate(w)
+    q, k, v = q.to(dev()), k.to(dev()), v.to(dev())
+    idx, ws = run_select(q, k, params)
+    heads = list(range(w.h_q))
+    sels = PT.oracle_select_heads(q, k, params, heads)
+    nb = w.n // 128
+    PT.compare_selection(idx, sels, nb)
+    G = w.h_q // w.h_kv
+    if params.route_rule:
+        for h in heads:
+            assert int(idx.route[h]) == int(meta["concentrated"][h]), (h, float(idx.debug[h, 2 * nb + 4]))
+    o, lse = crisp.sparse_prefill(q, k, v, idx, ws=ws)
+    crisp.check_status(ws)
+    ah = [0, 2, w.h_q - 1]
+    PT.assert_attention_ok(PT.compare_attention_blocks(q, k, v, o, lse, all_lists(idx, ah),
+                                                       sample_blocks(nb, ah, 3, seed=n), G))
+
+
+def test_flexprefill_full_128k():
+    """The baseline rules at the 128k Llama geometry: routes follow the planted structure, and
+    the gamma rule collapses sink-dominated Vertical-Slash heads onto their anchors."""
+    w = W.WORKLOADS["llama8b_128k"]
+    q, k, v, meta = W.generate(w, device=dev())
+    params = crisp.Params.flexprefill()
+    ws = crisp.workspace(w.h_q, w.h_kv, w.n, dev())
+    idx = crisp.Index.empty(w.h_q, w.n, dev(), debug=True)
+    o, lse, idx = crisp.prefill(q, k, v, params, index=idx, ws=ws)
+    crisp.check_status(ws)
+    nb = w.n // 128
+    heads = [0, 1, 2, 3, 12, 13, 30, 31]
+    sels = PT.oracle_select_heads(q, k, params, heads)
+    PT.compare_selection(idx, sels, nb)
+    for h in range(w.h_q):
+        assert int(idx.route[h]) == int(meta["concentrated"][h])
+    PT.assert_attention_ok(PT.compare_attention_blocks(q, k, v, o, lse, all_lists(idx, [0, 2]),
+                                                       sample_blocks(nb, [0, 2], 1, seed=3), w.h_q // w.h_kv))
+
+
 # ------------------------------------------------------------------------------ full-size workloads
 def _full(name, sel_heads, attn_per_head, attn_heads=None, seed=0):
     w = W.WORKLOADS[name]
