@@ -53,6 +53,20 @@ def dist_env():
     return world, rank, local
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's time: every rank takes part, in the same order, so ranks never diverge."""
+    if world <= 1:
+        return x
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, n: int, steps: int, total_s: float) -> float:
+    """Whole-job throughput: every rank processes `steps` layers of n tokens in the slowest rank's time."""
+    return world * n * steps / total_s
+
+
 class ClockSampler:
     """nvidia-smi clock/throttle sampling during the timed region."""
 
@@ -226,11 +240,7 @@ def run_crisp(args):
     t_att = np.array([ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]) / 1e3
     t_step = t_sel + t_att
     total_s = float(t_step.sum())
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([total_s], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_s = float(tt.item())
+    total_s = max_over_ranks(total_s, world, dev)
 
     # end to end through the public API: pinned host inputs -> device, prefill, output -> host
     e2e = None
@@ -254,14 +264,10 @@ def run_crisp(args):
         torch.cuda.synchronize()
         crisp.check_status(ws, "e2e")
         e2e_s = e0.elapsed_time(e1) / 1e3 / e_steps
-        if world > 1:
-            import torch.distributed as dist
-            tt = torch.tensor([e2e_s], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_s = float(tt.item())
+        e2e_s = max_over_ranks(e2e_s, world, dev)
         h2d = (q.numel() + k.numel() + v.numel()) * 2
         d2h = o.numel() * 2
-        e2e = {"value": world * w.n / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": job_tokens_per_s(world, w.n, 1, e2e_s), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_s * 1e3}
 
     if rank != 0:
@@ -279,7 +285,7 @@ def run_crisp(args):
     dense_pairs = w.h_q * nb * (nb + 1) // 2
     out = {
         "metric": METRIC,
-        "value": world * w.n * args.steps / total_s,
+        "value": job_tokens_per_s(world, w.n, args.steps, total_s),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
