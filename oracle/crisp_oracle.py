@@ -36,6 +36,8 @@ Readings where the pages leave a step open (each also listed in the design notes
      blocks are added as for CRISP (the merge of R6 is unchanged);
   R10 (median floor, [CRISP] §4 robustness discussion / Table 9) mu_d is the median of
      p_d[1..N_b-2] (mean of the two middle values when N_b-2 is even); the keep rule is unchanged.
+  R11 (attention at any length) with n not a multiple of B there are N_b = ceil(n/B) blocks and
+     the last query and key blocks are partial; a block's keys are its tokens below n.
 """
 from __future__ import annotations
 
@@ -325,8 +327,10 @@ def attention_block(q_blk: np.ndarray, k: np.ndarray, v: np.ndarray, key_blocks,
     Returns (O [B, d], lse [B]) with lse the natural-log sum of exp of the scaled logits.
     """
     d = q_blk.shape[1]
-    keys = np.concatenate([np.arange(kb * B, kb * B + B) for kb in key_blocks])
-    rows = np.arange(qb * B, qb * B + B)
+    n = k.shape[0]
+    # the last block of a sequence whose length is not a multiple of B is partial (R11)
+    keys = np.concatenate([np.arange(kb * B, min(kb * B + B, n)) for kb in key_blocks])
+    rows = np.arange(qb * B, qb * B + q_blk.shape[0])
     s = (q_blk @ k[keys].T) / np.sqrt(d)
     allowed = keys[None, :] <= rows[:, None]
     s = np.where(allowed, s, -np.inf)

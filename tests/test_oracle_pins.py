@@ -58,10 +58,11 @@ def test_attention_bruteforce_loop_tiny():
         assert abs(lse[i] - (mx + math.log(z))) < 1e-12
 
 
-@pytest.mark.parametrize("n", [128, 256, 512, 1024])
+@pytest.mark.parametrize("n", [128, 256, 512, 1024, 1, 77, 129, 300, 1000])
 def test_all_blocks_equals_sdpa_dense(n):
+    # lengths that are not a multiple of 128 have a partial last block (R11)
     q, k, v = (f64(t[0]) for t in W.random_qkv(1, 1, n, seed=n))
-    lists = [np.arange(qb + 1) for qb in range(n // 128)]
+    lists = [np.arange(qb + 1) for qb in range(-(-n // 128))]
     o, _ = O.attention_head(q, k, v, lists)
     ref = sdpa_masked(q, k, v, np.tril(np.ones((n, n), dtype=bool)))
     assert np.max(np.abs(o - ref)) < 1e-12
