@@ -151,7 +151,11 @@ def _qkv_shape(q, k, v=None):
 
 
 def workspace_size(h_q: int, h_kv: int, n: int, d: int = 128, params: Params | None = None) -> int:
-    p = (params or Params()).c()
+    """Workspace bytes for this shape; without params any length counts (attention alone runs at
+    any n, selection needs a multiple of 128)."""
+    if params is None:
+        return int(lib().crisp_workspace_size(h_q, h_kv, n, d, None))
+    p = params.c()
     return int(lib().crisp_workspace_size(h_q, h_kv, n, d, ctypes.byref(p)))
 
 

@@ -39,12 +39,28 @@ int make_map(CUtensorMap* m, const void* base, uint64_t rows) {
   return r == CUDA_SUCCESS ? CRISP_OK : CRISP_ERR_CUDA;
 }
 
+// 3D bf16 view [heads][n][128] with 64x128x1 boxes: a head's rows past n read as zeros, so a
+// partial last block never sees the next head's rows.
+int make_map3(CUtensorMap* m, const void* base, uint64_t n, uint64_t heads) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return CRISP_ERR_CUDA;
+  cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)n, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)kD * 2 * n};
+  cuuint32_t box[3] = {64, (cuuint32_t)kB, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? CRISP_OK : CRISP_ERR_CUDA;
+}
+
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-int check_shape(int h_q, int h_kv, int n, int d, Shape* s) {
+// Attention runs at any n (a partial last block); selection needs n to be a multiple of 128.
+int check_shape(int h_q, int h_kv, int n, int d, Shape* s, bool any_length = false) {
   if (h_q <= 0 || h_kv <= 0 || n <= 0 || d <= 0) return CRISP_ERR_INVALID_ARG;
-  if (d != kD || n % kB != 0 || h_q % h_kv != 0) return CRISP_ERR_UNSUPPORTED;
-  const long long nb = n / kB;
+  if (d != kD || h_q % h_kv != 0 || (!any_length && n % kB != 0)) return CRISP_ERR_UNSUPPORTED;
+  const long long nb = (n + kB - 1) / kB;
   const long long cap = nb * (nb + 1) / 2;
   if (cap > 0x7fffffffLL || (long long)h_q * n > 0x7fffffffLL || (long long)h_kv * n > 0x7fffffffLL)
     return CRISP_ERR_OVERFLOW;
@@ -161,9 +177,9 @@ int run_attention(const void* q, const void* k, const void* v, const Shape& s, c
   a.trace = at<unsigned long long>(ws, w.trace);
   a.scale_log2 = 0.12751743074380045f;  // log2(e) / sqrt(128)
   CUtensorMap qm, km, vm;
-  int rc = make_map(&qm, q, (uint64_t)s.h_q * s.n);
-  if (rc == CRISP_OK) rc = make_map(&km, k, (uint64_t)s.h_kv * s.n);
-  if (rc == CRISP_OK) rc = make_map(&vm, v, (uint64_t)s.h_kv * s.n);
+  int rc = make_map3(&qm, q, (uint64_t)s.n, (uint64_t)s.h_q);
+  if (rc == CRISP_OK) rc = make_map3(&km, k, (uint64_t)s.n, (uint64_t)s.h_kv);
+  if (rc == CRISP_OK) rc = make_map3(&vm, v, (uint64_t)s.n, (uint64_t)s.h_kv);
   if (rc != CRISP_OK) return rc;
   return launch_sparse_attn(qm, km, vm, a, st) == cudaSuccess ? CRISP_OK : CRISP_ERR_CUDA;
 }
@@ -197,7 +213,7 @@ extern "C" {
 
 size_t crisp_workspace_size(int h_q, int h_kv, int n, int d, const crisp_params* params) {
   Shape s;
-  if (check_shape(h_q, h_kv, n, d, &s) != CRISP_OK) return 0;
+  if (check_shape(h_q, h_kv, n, d, &s, params == nullptr) != CRISP_OK) return 0;
   if (params != nullptr && check_params(params) != CRISP_OK) return 0;
   return workspace_layout(s).total;
 }
@@ -218,7 +234,7 @@ int crisp_select(const void* q, const void* k, int h_q, int h_kv, int n, int d, 
 int crisp_sparse_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv, int n, int d,
                          const crisp_index* idx, void* o, float* lse, void* ws, size_t ws_bytes, void* stream) {
   Shape s;
-  int rc = check_shape(h_q, h_kv, n, d, &s);
+  int rc = check_shape(h_q, h_kv, n, d, &s, true);
   if (rc == CRISP_OK && (!tensors_ok(q, k, v) || v == nullptr || o == nullptr || !aligned(o, 16)))
     rc = CRISP_ERR_INVALID_ARG;
   if (rc == CRISP_OK) rc = check_index(idx, false);
@@ -260,7 +276,7 @@ int crisp_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv
 int crisp_dense_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv, int n, int d, void* o,
                         float* lse, void* ws, size_t ws_bytes, void* stream) {
   Shape s;
-  int rc = check_shape(h_q, h_kv, n, d, &s);
+  int rc = check_shape(h_q, h_kv, n, d, &s, true);
   if (rc == CRISP_OK && (!tensors_ok(q, k, v) || v == nullptr || o == nullptr || !aligned(o, 16)))
     rc = CRISP_ERR_INVALID_ARG;
   if (rc == CRISP_OK) rc = check_ws(ws, ws_bytes, s);

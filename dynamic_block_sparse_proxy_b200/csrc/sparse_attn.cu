@@ -21,6 +21,9 @@
 //               (A operand read from TMEM), then S_t = Q_t K^T of this step; the two tiles run
 //               out of phase, so the tensor core works on one while the other's softmax runs.
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; P_t is packed bf16 over S_t.
+// Q, K and V are read through per-head 3D tensor maps: when n is not a multiple of 128 the last
+// block's rows past n arrive as zeros; the causal mask already hides keys past n from every
+// real query (key j <= query i < n), and output rows past n are not stored.
 // tcgen05 MMAs issued by one thread execute in order, so S_t is overwritten only after the PV
 // that read P_t from the same columns, and the commit that signals S_t also covers that PV.
 // Both tiles' MMAs run on the same tensor core, interleaved as their issuers go.
@@ -239,21 +242,21 @@ __global__ void __launch_bounds__(THREADS, 1)
       tma_prefetch_desc(&k_map);
       mbar_arrive_expect_tx(&sm.q_full, TILE_BYTES * ntiles);
       for (int t = 0; t < ntiles; ++t) {
-        const int qrow = (t ? tile_h[1] : tile_h[0]) * s.n + (t ? tile_qb[1] : tile_qb[0]) * kB;
-        tma_load_2d(&q_map, &sm.q_full, sm.q[t], 0, qrow);
-        tma_load_2d(&q_map, &sm.q_full, sm.q[t] + kB * 64, 64, qrow);
+        const int qh = t ? tile_h[1] : tile_h[0], qy = (t ? tile_qb[1] : tile_qb[0]) * kB;
+        tma_load_3d(&q_map, &sm.q_full, sm.q[t], 0, qy, qh);
+        tma_load_3d(&q_map, &sm.q_full, sm.q[t] + kB * 64, 64, qy, qh);
       }
       UnionWalk u(tl, dense, tile_qb);
       int kb, mask, nk = 0;
       for (int step = 0; u.next(kb, mask); ++step) {
         const int st = step % NSK;
         const uint32_t par = ((step / NSK) & 1) ^ 1;
-        const int krow = kv * s.n + kb * kB;
+        const int ky = kb * kB;
         trace_mark(a.trace, 0, 0, 1, step);
         if (!mbar_wait(&sm.k_empty[st], par, abort)) { fail(sm, a.status, CRISP_ERR_DEVICE_TIMEOUT); break; }
         mbar_arrive_expect_tx(&sm.k_full[st], TILE_BYTES);
-        tma_load_2d(&k_map, &sm.k_full[st], sm.k[st], 0, krow);
-        tma_load_2d(&k_map, &sm.k_full[st], sm.k[st] + kB * 64, 64, krow);
+        tma_load_3d(&k_map, &sm.k_full[st], sm.k[st], 0, ky, kv);
+        tma_load_3d(&k_map, &sm.k_full[st], sm.k[st] + kB * 64, 64, ky, kv);
         nk = step + 1;
       }
       if (u.bad) record_status(a.status, CRISP_ERR_DEVICE_CHECK);
@@ -274,12 +277,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int step = 0; u.next(kb, mask); ++step) {
         const int st = step % NSV;
         const uint32_t par = ((step / NSV) & 1) ^ 1;
-        const int krow = kv * s.n + kb * kB;
+        const int ky = kb * kB;
         trace_mark(a.trace, 0, 5, 2, step);
         if (!mbar_wait(&sm.v_empty[st], par, abort)) { fail(sm, a.status, CRISP_ERR_DEVICE_TIMEOUT); break; }
         mbar_arrive_expect_tx(&sm.v_full[st], TILE_BYTES);
-        tma_load_2d(&v_map, &sm.v_full[st], sm.v[st], 0, krow);
-        tma_load_2d(&v_map, &sm.v_full[st], sm.v[st] + kB * 64, 64, krow);
+        tma_load_3d(&v_map, &sm.v_full[st], sm.v[st], 0, ky, kv);
+        tma_load_3d(&v_map, &sm.v_full[st], sm.v[st] + kB * 64, 64, ky, kv);
         nv = step + 1;
       }
       for (int i = max(0, nv - NSV); i < nv; ++i) mbar_wait(&sm.v_full[i % NSV], (i / NSV) & 1, nullptr);
@@ -502,6 +505,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         const float inv = 1.f / l;
         const size_t row = (size_t)my_h * s.n + (size_t)my_qb * kB + r;
+        const bool real = my_qb * kB + r < s.n;  // rows past n of a partial last block are not stored
         uint4* dst = reinterpret_cast<uint4*>(a.o + row * kD);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -510,14 +514,15 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            dst[c * 4 + j] = make_uint4(
+            if (real)
+              dst[c * 4 + j] = make_uint4(
                 pack_bf16(__uint_as_float(o[8 * j + 0]) * inv, __uint_as_float(o[8 * j + 1]) * inv),
                 pack_bf16(__uint_as_float(o[8 * j + 2]) * inv, __uint_as_float(o[8 * j + 3]) * inv),
                 pack_bf16(__uint_as_float(o[8 * j + 4]) * inv, __uint_as_float(o[8 * j + 5]) * inv),
                 pack_bf16(__uint_as_float(o[8 * j + 6]) * inv, __uint_as_float(o[8 * j + 7]) * inv));
           }
         }
-        if (a.lse != nullptr) a.lse[row] = (m + __log2f(l)) * kLn2;
+        if (a.lse != nullptr && real) a.lse[row] = (m + __log2f(l)) * kLn2;
         if (tracer) trace_mark(a.trace, 0, role, 6, L);
       }
     }

@@ -88,6 +88,16 @@ def test_select_rejects_bad_arguments_before_launch(L):
         assert rc in (-1, -2), bad
 
 
+def test_lengths_not_multiple_of_128(L):
+    # attention runs at any length (workspace sized without params); selection does not
+    p = crisp.Params().c()
+    assert L.crisp_workspace_size(2, 1, 1000, 128, None) > 0
+    assert L.crisp_workspace_size(2, 1, 1000, 128, ctypes.byref(p)) == 0
+    ix = _idx()
+    assert L.crisp_select(0x10000, 0x10000, 2, 1, 1000, 128, ctypes.byref(p), ctypes.byref(ix), 0x100000,
+                          1 << 40, None) == -2
+
+
 def test_selection_beyond_8192_blocks_is_unsupported(L):
     p = crisp.Params().c()
     ix = _idx()
@@ -106,7 +116,8 @@ def test_attention_entry_points_reject_bad_arguments(L):
                                   None) == -1
     assert L.crisp_sparse_prefill(fake, fake, fake, 1, 1, 4096, 128, ctypes.byref(ix), None, None, ws, big, None) == -1
     assert L.crisp_sparse_prefill(fake, fake, fake, 1, 1, 4096, 128, ctypes.byref(ix), fake, None, ws, 10, None) == -3
-    assert L.crisp_dense_prefill(fake, fake, fake, 1, 1, 4100, 128, fake, None, ws, big, None) == -2
+    # (fake pointers only with arguments refused before any launch)
+    assert L.crisp_dense_prefill(fake, fake, fake, 1, 1, 4096, 64, fake, None, ws, big, None) == -2
     assert L.crisp_dense_prefill(fake, fake, fake, 2, 4, 4096, 128, fake, None, ws, big, None) == -2
     p = crisp.Params().c()
     assert L.crisp_prefill(fake, fake, fake, 1, 1, 4096, 128, ctypes.byref(p), fake, None, None, ws, 10, None) == -3

@@ -64,13 +64,14 @@ def test_timeout_selftest_reports_and_context_survives():
     assert np.max(np.abs(PT.f64(o[0]) - ref)) < 2e-2
 
 
-@pytest.mark.parametrize("n,hq,hkv", [(128, 1, 1), (256, 2, 1), (384, 1, 1), (640, 3, 1), (896, 7, 1), (1024, 4, 2)])
+@pytest.mark.parametrize("n,hq,hkv", [(128, 1, 1), (256, 2, 1), (384, 1, 1), (640, 3, 1), (896, 7, 1), (1024, 4, 2),
+                                        (1, 1, 1), (77, 2, 1), (129, 3, 1), (300, 4, 2), (1000, 7, 1), (4097, 8, 2)])
 def test_dense_matches_oracle(n, hq, hkv):
     q, k, v = (t.to(dev()) for t in W.random_qkv(hq, hkv, n, seed=n + hq))
     ws = crisp.workspace(hq, hkv, n, dev())
     o, lse = crisp.dense_prefill(q, k, v, ws=ws)
     crisp.check_status(ws)
-    nb = n // 128
+    nb = -(-n // 128)  # a length that is not a multiple of 128 ends in a partial block
     lists = {h: [list(range(qb + 1)) for qb in range(nb)] for h in range(hq)}
     blocks = [(h, qb) for h in range(hq) for qb in range(nb)]
     PT.assert_attention_ok(PT.compare_attention_blocks(q, k, v, o, lse, lists, blocks, hq // hkv))
@@ -173,12 +174,13 @@ def test_pe_uniform_closed_form_on_gpu():
 
 
 @pytest.mark.parametrize("n,hq,hkv,mixed", [(2048, 4, 2, False), (1152, 3, 1, False), (640, 1, 1, False),
-                                            (1920, 14, 2, True), (1152, 5, 1, True)])
+                                            (1920, 14, 2, True), (1152, 5, 1, True), (1000, 4, 2, True),
+                                            (2177, 3, 1, False)])
 def test_user_index_through_sparse_prefill(n, hq, hkv, mixed):
     # random strictly ascending lists with the diagonal block; odd group sizes and odd block
     # counts pair a head's adjacent query blocks in one CTA
     q, k, v = (t.to(dev()) for t in W.random_qkv(hq, hkv, n, seed=5))
-    nb = n // 128
+    nb = -(-n // 128)  # partial last block when n is not a multiple of 128
     rng = np.random.default_rng(9)
     cap = nb * (nb + 1) // 2
     row_ptr = np.zeros((hq, nb + 1), dtype=np.int32)
