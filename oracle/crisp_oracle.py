@@ -36,8 +36,10 @@ Readings where the pages leave a step open (each also listed in the design notes
      blocks are added as for CRISP (the merge of R6 is unchanged);
   R10 (median floor, [CRISP] §4 robustness discussion / Table 9) mu_d is the median of
      p_d[1..N_b-2] (mean of the two middle values when N_b-2 is even); the keep rule is unchanged.
-  R11 (attention at any length) with n not a multiple of B there are N_b = ceil(n/B) blocks and
-     the last query and key blocks are partial; a block's keys are its tokens below n.
+  R11 (any length) with n not a multiple of B there are N_b = ceil(n/B) blocks and the last
+     query and key blocks are partial: a block's keys are its tokens below n, block masses pool
+     what the block has, block means average the rows it has; the proxy still takes the last B
+     queries and the anchors are still the first and last B keys (selection needs n >= B).
 """
 from __future__ import annotations
 
@@ -98,10 +100,16 @@ def jsd(p: np.ndarray, q: np.ndarray) -> float:
 # ----------------------------------------------------------------------------------------------
 # Vertical and slash scores pooled into key blocks  ([CRISP] §4, decomposition paragraph)
 # ----------------------------------------------------------------------------------------------
+def pool_blocks(x: np.ndarray, B: int) -> np.ndarray:
+    """Sums of consecutive runs of B entries; a partial last run sums what exists (R11)."""
+    nb = -(-x.shape[0] // B)
+    return np.concatenate([x, np.zeros(nb * B - x.shape[0])]).reshape(nb, B).sum(axis=1)
+
+
 def vertical_block_mass(a_hat: np.ndarray, B: int) -> np.ndarray:
     """p_v[b] = sum over keys of block b of the column mean of A_hat (R3)."""
     col_mean = a_hat.mean(axis=0)                             # (1/B) sum_r
-    return col_mean.reshape(-1, B).sum(axis=1)
+    return pool_blocks(col_mean, B)
 
 
 def slash_block_mass(a_hat: np.ndarray, n: int, B: int) -> np.ndarray:
@@ -115,7 +123,7 @@ def slash_block_mass(a_hat: np.ndarray, n: int, B: int) -> np.ndarray:
         # offsets 0..i_r read the row backwards from the diagonal
         a_s[: i_r + 1] += a_hat[r, i_r::-1]
     a_s /= B
-    return a_s.reshape(-1, B).sum(axis=1)
+    return pool_blocks(a_s, B)
 
 
 # ----------------------------------------------------------------------------------------------
@@ -187,8 +195,10 @@ def merge_vertical_slash(keep_v, keep_s, nb: int) -> list[np.ndarray]:
 # Pooled-Estimation path  ([CRISP] §2 and §4 PE paragraph; [BLOG] gamma_cumsum(pool(Q), pool(K)))
 # ----------------------------------------------------------------------------------------------
 def block_mean(x: np.ndarray, B: int) -> np.ndarray:
-    """Mean of each block of B consecutive rows: [n, d] -> [n/B, d]."""
-    return x.reshape(-1, B, x.shape[1]).mean(axis=1)
+    """Mean of each block of B consecutive rows: [n, d] -> [ceil(n/B), d]; a partial last block
+    is the mean of the rows it has (R11)."""
+    n = x.shape[0]
+    return np.stack([x[i:min(i + B, n)].mean(axis=0) for i in range(0, n, B)])
 
 
 def pooled_scores(q: np.ndarray, k: np.ndarray, B: int) -> np.ndarray:
@@ -266,7 +276,7 @@ def select_head(q: np.ndarray, k: np.ndarray, *, block=128, anchors=128, tau_pro
     """
     n = q.shape[0]
     B = block
-    nb = n // B
+    nb = -(-n // B)                     # partial last block when n is not a multiple of B (R11)
     a_hat = proxy_attention(q[n - B:], k, n)
     c = c_struct(a_hat, n, anchors)
     p_v = vertical_block_mass(a_hat, B)
