@@ -120,7 +120,7 @@ class ClockSampler:
 def select_bytes(w, n_pe_heads: int, total_pairs: int) -> float:
     """Algorithmic HBM bytes of selection: K once, the last query block of every head, the
     whole Q of the Pooled-Estimation heads, and the written index (row_ptr + cols)."""
-    nb = w.n // 128
+    nb = -(-w.n // 128)
     k_bytes = w.h_kv * w.n * w.d * 2
     qlast = w.h_q * 128 * w.d * 2
     qpe = n_pe_heads * w.n * w.d * 2
@@ -215,7 +215,7 @@ def run_crisp(args):
         flush.fill_(1)
         step()
     crisp.check_status(ws, "warmup")
-    nb = w.n // 128
+    nb = -(-w.n // 128)
     total_pairs = int(idx.row_ptr[:, nb].sum().item())
     n_pe = int((idx.route == 0).sum().item())
 
@@ -327,7 +327,7 @@ def oracle_baseline(w, q, k, v, idx, budget_s: float, seed: int = 0, params=None
     from oracle import crisp_oracle as O
 
     G = w.h_q // w.h_kv
-    nb = w.n // 128
+    nb = -(-w.n // 128)
     route = idx.route.cpu().numpy() if idx is not None else None
     conc = W.concentrated_heads(w)
     # one head of each kind the workload has (a one-head workload has only one)

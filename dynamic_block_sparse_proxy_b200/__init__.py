@@ -111,11 +111,27 @@ class Index:
 
     @staticmethod
     def empty(h_q: int, n: int, device, debug: bool = False) -> "Index":
-        nb = n // 128
+        nb = n_blocks(n)
         i32 = dict(device=device, dtype=torch.int32)
         return Index(torch.empty(h_q, **i32), torch.empty(h_q, device=device, dtype=torch.float32),
                      torch.empty(h_q, nb + 1, **i32), torch.empty(h_q, nb * (nb + 1) // 2, **i32),
                      torch.empty(h_q, 2 * nb + 5, device=device, dtype=torch.float32) if debug else None)
+
+    def check(self, h_q: int, n: int, need_select_fields: bool = True):
+        """Raise unless every array is a contiguous device tensor large enough for (h_q, n): the
+        library writes and reads these sizes without seeing the tensors."""
+        nb = n_blocks(n)
+        want = [("row_ptr", self.row_ptr, torch.int32, (h_q, nb + 1)),
+                ("cols", self.cols, torch.int32, (h_q, nb * (nb + 1) // 2))]
+        if need_select_fields:
+            want += [("route", self.route, torch.int32, (h_q,)), ("c_struct", self.c_struct, torch.float32, (h_q,))]
+        elif self.route is not None:  # attention reads it to schedule heads
+            want.append(("route", self.route, torch.int32, (h_q,)))
+            if self.debug is not None:
+                want.append(("debug", self.debug, torch.float32, (h_q, 2 * nb + 5)))
+        for name, t, dt, shape in want:
+            if t is None or not t.is_cuda or t.dtype != dt or not t.is_contiguous() or tuple(t.shape) != shape:
+                raise ValueError(f"index.{name} must be a contiguous {dt} CUDA tensor of shape {shape}")
 
     def c(self) -> _Index:
         return _Index(self.route.data_ptr(), self.c_struct.data_ptr(), self.row_ptr.data_ptr(),
@@ -126,6 +142,19 @@ class Index:
         rp = self.row_ptr[h].cpu().tolist()
         cols = self.cols[h].cpu()
         return [cols[rp[i]:rp[i + 1]].tolist() for i in range(len(rp) - 1)]
+
+
+def n_blocks(n: int) -> int:
+    """Number of 128-token blocks; a length that is not a multiple of 128 ends in a partial block."""
+    return -(-n // 128)
+
+
+def _check_out(q, o, lse):
+    if not o.is_cuda or o.dtype != torch.bfloat16 or not o.is_contiguous() or o.shape != q.shape:
+        raise ValueError("o must be a contiguous bf16 CUDA tensor shaped like q")
+    if lse is not None and (not lse.is_cuda or lse.dtype != torch.float32 or not lse.is_contiguous()
+                            or tuple(lse.shape) != (q.shape[0], q.shape[1])):
+        raise ValueError("lse must be a contiguous fp32 CUDA tensor of shape [h_q, n]")
 
 
 def _check(code: int, where: str):
@@ -174,6 +203,7 @@ def select(q, k, params: Params | None = None, index: Index | None = None, ws: t
     params = params or Params()
     ws = ws if ws is not None else workspace(h_q, h_kv, n, q.device, d)
     index = index or Index.empty(h_q, n, q.device, debug=debug)
+    index.check(h_q, n)
     p, ix = params.c(), index.c()
     _check(lib().crisp_select(q.data_ptr(), k.data_ptr(), h_q, h_kv, n, d, ctypes.byref(p), ctypes.byref(ix),
                               ws.data_ptr(), ws.numel(), _stream(q)), "crisp_select")
@@ -187,6 +217,8 @@ def sparse_prefill(q, k, v, index: Index, o=None, lse=None, ws=None, want_lse: b
     o = o if o is not None else torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty(h_q, n, device=q.device, dtype=torch.float32)
+    _check_out(q, o, lse)
+    index.check(h_q, n, need_select_fields=False)
     ix = index.c()
     _check(lib().crisp_sparse_prefill(q.data_ptr(), k.data_ptr(), v.data_ptr(), h_q, h_kv, n, d, ctypes.byref(ix),
                                       o.data_ptr(), lse.data_ptr() if lse is not None else None, ws.data_ptr(),
@@ -205,6 +237,9 @@ def prefill(q, k, v, params: Params | None = None, index: Index | None = None, o
         lse = torch.empty(h_q, n, device=q.device, dtype=torch.float32)
     if index is None and keep_index:
         index = Index.empty(h_q, n, q.device)
+    _check_out(q, o, lse)
+    if index is not None:
+        index.check(h_q, n)
     p = params.c()
     ix = ctypes.byref(index.c()) if index is not None else None
     _check(lib().crisp_prefill(q.data_ptr(), k.data_ptr(), v.data_ptr(), h_q, h_kv, n, d, ctypes.byref(p),
@@ -220,6 +255,7 @@ def dense_prefill(q, k, v, o=None, lse=None, ws=None, want_lse: bool = True):
     o = o if o is not None else torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty(h_q, n, device=q.device, dtype=torch.float32)
+    _check_out(q, o, lse)
     _check(lib().crisp_dense_prefill(q.data_ptr(), k.data_ptr(), v.data_ptr(), h_q, h_kv, n, d, o.data_ptr(),
                                      lse.data_ptr() if lse is not None else None, ws.data_ptr(), ws.numel(),
                                      _stream(q)), "crisp_dense_prefill")

@@ -25,20 +25,6 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2D bf16 view [rows][128] with 64x128 boxes and 128-byte swizzle.
-int make_map(CUtensorMap* m, const void* base, uint64_t rows) {
-  auto fn = encode_fn();
-  if (fn == nullptr) return CRISP_ERR_CUDA;
-  cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)kB};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? CRISP_OK : CRISP_ERR_CUDA;
-}
-
 // 3D bf16 view [heads][n][128] with 64x128x1 boxes: a head's rows past n read as zeros, so a
 // partial last block never sees the next head's rows.
 int make_map3(CUtensorMap* m, const void* base, uint64_t n, uint64_t heads) {
@@ -56,10 +42,10 @@ int make_map3(CUtensorMap* m, const void* base, uint64_t n, uint64_t heads) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-// Attention runs at any n (a partial last block); selection needs n to be a multiple of 128.
-int check_shape(int h_q, int h_kv, int n, int d, Shape* s, bool any_length = false) {
+// Any n >= 1 (a partial last block when n is not a multiple of 128); selection adds n >= 128.
+int check_shape(int h_q, int h_kv, int n, int d, Shape* s) {
   if (h_q <= 0 || h_kv <= 0 || n <= 0 || d <= 0) return CRISP_ERR_INVALID_ARG;
-  if (d != kD || h_q % h_kv != 0 || (!any_length && n % kB != 0)) return CRISP_ERR_UNSUPPORTED;
+  if (d != kD || h_q % h_kv != 0) return CRISP_ERR_UNSUPPORTED;
   const long long nb = (n + kB - 1) / kB;
   const long long cap = nb * (nb + 1) / 2;
   if (cap > 0x7fffffffLL || (long long)h_q * n > 0x7fffffffLL || (long long)h_kv * n > 0x7fffffffLL)
@@ -126,6 +112,8 @@ int run_select(const void* q, const void* k, const Shape& s, const crisp_params*
   a.pv = at<double>(ws, w.pv);
   a.ps_lo = at<double>(ws, w.ps_lo);
   a.ps_hi = at<double>(ws, w.ps_hi);
+  a.ps_x = at<double>(ws, w.ps_x);
+  a.rec_extra = at<float>(ws, w.rec_extra);
   a.kbar = at<float>(ws, w.kbar);
   a.qbar = at<float>(ws, w.qbar);
   a.pbuf = at<float>(ws, w.pbuf);
@@ -145,8 +133,8 @@ int run_select(const void* q, const void* k, const Shape& s, const crisp_params*
   a.debug = out.debug;
 
   CUtensorMap qm, km;
-  int rc = make_map(&qm, q, (uint64_t)s.h_q * s.n);
-  if (rc == CRISP_OK) rc = make_map(&km, k, (uint64_t)s.h_kv * s.n);
+  int rc = make_map3(&qm, q, (uint64_t)s.n, (uint64_t)s.h_q);
+  if (rc == CRISP_OK) rc = make_map3(&km, k, (uint64_t)s.n, (uint64_t)s.h_kv);
   if (rc != CRISP_OK) return rc;
 
   // The radix histograms accumulate with atomics: start from zero.
@@ -213,7 +201,8 @@ extern "C" {
 
 size_t crisp_workspace_size(int h_q, int h_kv, int n, int d, const crisp_params* params) {
   Shape s;
-  if (check_shape(h_q, h_kv, n, d, &s, params == nullptr) != CRISP_OK) return 0;
+  if (check_shape(h_q, h_kv, n, d, &s) != CRISP_OK) return 0;
+  if (params != nullptr && n < kB) return 0;
   if (params != nullptr && check_params(params) != CRISP_OK) return 0;
   return workspace_layout(s).total;
 }
@@ -223,7 +212,7 @@ int crisp_select(const void* q, const void* k, int h_q, int h_kv, int n, int d, 
   Shape s;
   int rc = check_shape(h_q, h_kv, n, d, &s);
   if (rc == CRISP_OK) rc = check_params(params);
-  if (rc == CRISP_OK && s.nb > kMaxSelectBlocks) rc = CRISP_ERR_UNSUPPORTED;
+  if (rc == CRISP_OK && (s.nb > kMaxSelectBlocks || n < kB)) rc = CRISP_ERR_UNSUPPORTED;
   if (rc == CRISP_OK && !tensors_ok(q, k, nullptr)) rc = CRISP_ERR_INVALID_ARG;
   if (rc == CRISP_OK) rc = check_index(out, true);
   if (rc == CRISP_OK) rc = check_ws(ws, ws_bytes, s);
@@ -234,7 +223,7 @@ int crisp_select(const void* q, const void* k, int h_q, int h_kv, int n, int d, 
 int crisp_sparse_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv, int n, int d,
                          const crisp_index* idx, void* o, float* lse, void* ws, size_t ws_bytes, void* stream) {
   Shape s;
-  int rc = check_shape(h_q, h_kv, n, d, &s, true);
+  int rc = check_shape(h_q, h_kv, n, d, &s);
   if (rc == CRISP_OK && (!tensors_ok(q, k, v) || v == nullptr || o == nullptr || !aligned(o, 16)))
     rc = CRISP_ERR_INVALID_ARG;
   if (rc == CRISP_OK) rc = check_index(idx, false);
@@ -250,7 +239,7 @@ int crisp_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv
   Shape s;
   int rc = check_shape(h_q, h_kv, n, d, &s);
   if (rc == CRISP_OK) rc = check_params(params);
-  if (rc == CRISP_OK && s.nb > kMaxSelectBlocks) rc = CRISP_ERR_UNSUPPORTED;
+  if (rc == CRISP_OK && (s.nb > kMaxSelectBlocks || n < kB)) rc = CRISP_ERR_UNSUPPORTED;
   if (rc == CRISP_OK && (!tensors_ok(q, k, v) || v == nullptr || o == nullptr || !aligned(o, 16)))
     rc = CRISP_ERR_INVALID_ARG;
   if (rc == CRISP_OK && idx_out != nullptr) rc = check_index(idx_out, true);
@@ -276,7 +265,7 @@ int crisp_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv
 int crisp_dense_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv, int n, int d, void* o,
                         float* lse, void* ws, size_t ws_bytes, void* stream) {
   Shape s;
-  int rc = check_shape(h_q, h_kv, n, d, &s, true);
+  int rc = check_shape(h_q, h_kv, n, d, &s);
   if (rc == CRISP_OK && (!tensors_ok(q, k, v) || v == nullptr || o == nullptr || !aligned(o, 16)))
     rc = CRISP_ERR_INVALID_ARG;
   if (rc == CRISP_OK) rc = check_ws(ws, ws_bytes, s);

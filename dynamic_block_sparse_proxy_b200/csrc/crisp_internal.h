@@ -37,7 +37,8 @@ struct CutState {
 };
 
 struct Workspace {
-  size_t status, trace, part, chunk_max, chunk_tot, row_w, pv, ps_lo, ps_hi, kbar, qbar, pbuf, hist_cnt, hist_mass, cut,
+  size_t status, trace, part, chunk_max, chunk_tot, row_w, pv, ps_lo, ps_hi, ps_x, rec_extra, kbar, qbar, pbuf,
+      hist_cnt, hist_mass, cut,
       keep_v, keep_s, cnt, eqcnt, eqbase, idx_route, idx_c, idx_row_ptr, idx_cols, total;
 };
 
@@ -61,6 +62,8 @@ inline Workspace workspace_layout(const Shape& s) {
   w.pv = take(hq * nb * 8);
   w.ps_lo = take(hq * nb * 8);
   w.ps_hi = take(hq * nb * 8);
+  w.ps_x = take(hq * nb * 8);
+  w.rec_extra = take(hq * kB * 4);
   w.kbar = take((size_t)s.h_kv * nb * kD * 4);
   w.qbar = take(hq * nb * kD * 4);
   w.pbuf = take(hq * (size_t)s.cap * 4);
@@ -98,6 +101,8 @@ struct SelectArgs {
   double* pv;      // vertical block masses
   double* ps_lo;   // slash block masses from the keys at or below each row's diagonal offset
   double* ps_hi;   // ... and from the keys above it
+  double* ps_x;    // ... and (n not a multiple of 128) the next offset block down
+  float* rec_extra;  // per proxy row: recency-window mass inside block N_b-2 (n not a multiple of 128)
   float* kbar;
   float* qbar;
   float* pbuf;

@@ -47,15 +47,16 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
   return fn;
 }
 
-// bf16 [rows][128] with 64x128 boxes and 128-byte swizzle, as the selection kernels expect.
-int encode_rows(CUtensorMap* m, const void* base, uint64_t rows) {
+// bf16 [heads][n][128] with 64x128x1 boxes and 128-byte swizzle, as the selection kernels expect
+// (a head's rows past n read as zeros).
+int encode_heads(CUtensorMap* m, const void* base, uint64_t n, uint64_t heads) {
   auto fn = encode_tiled();
   if (fn == nullptr) return CRISP_ERR_CUDA;
-  cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)kB};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)n, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)kD * 2 * n};
+  cuuint32_t box[3] = {64, (cuuint32_t)kB, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS
              ? CRISP_OK
@@ -73,7 +74,7 @@ extern "C" int crisp_select_noalloc(const void* q, const void* k, int h_q, int h
                                     const crisp_params* p, const crisp_index* out, int* device_status,
                                     void* stream) {
   if (h_q <= 0 || h_kv <= 0 || n <= 0 || d <= 0 || p == nullptr || out == nullptr) return CRISP_ERR_INVALID_ARG;
-  if (d != kD || n % kB != 0 || h_q % h_kv != 0 || p->block != kB || p->anchors != kB) return CRISP_ERR_UNSUPPORTED;
+  if (d != kD || n < kB || h_q % h_kv != 0 || p->block != kB || p->anchors != kB) return CRISP_ERR_UNSUPPORTED;
   if (!std::isfinite(p->tau_proxy) || !std::isfinite(p->alpha) || !std::isfinite(p->gamma) || p->alpha < 0.f ||
       p->gamma <= 0.f || p->min_blocks < 0)
     return CRISP_ERR_INVALID_ARG;
@@ -81,7 +82,7 @@ extern "C" int crisp_select_noalloc(const void* q, const void* k, int h_q, int h
   if (out->route == nullptr || out->c_struct == nullptr || out->row_ptr == nullptr || out->cols == nullptr ||
       !is_aligned(out->row_ptr, 4) || !is_aligned(out->cols, 4))
     return CRISP_ERR_INVALID_ARG;
-  const long long nb = n / kB;
+  const long long nb = (n + kB - 1) / kB;  // a partial last block when n is not a multiple of 128
   const long long cap = nb * (nb + 1) / 2;
   if (cap > 0x7fffffffLL || (long long)h_q * n > 0x7fffffffLL) return CRISP_ERR_OVERFLOW;
   if (nb > kMaxSelectBlocks) return CRISP_ERR_UNSUPPORTED;
@@ -124,6 +125,8 @@ extern "C" int crisp_select_noalloc(const void* q, const void* k, int h_q, int h
   a.pv = reinterpret_cast<double*>(at(w.pv));
   a.ps_lo = reinterpret_cast<double*>(at(w.ps_lo));
   a.ps_hi = reinterpret_cast<double*>(at(w.ps_hi));
+  a.ps_x = reinterpret_cast<double*>(at(w.ps_x));
+  a.rec_extra = reinterpret_cast<float*>(at(w.rec_extra));
   a.kbar = reinterpret_cast<float*>(at(w.kbar));
   a.qbar = reinterpret_cast<float*>(at(w.qbar));
   a.pbuf = reinterpret_cast<float*>(at(w.pbuf));
@@ -143,8 +146,8 @@ extern "C" int crisp_select_noalloc(const void* q, const void* k, int h_q, int h
   a.debug = out->debug;
 
   CUtensorMap qm, km;
-  rc = encode_rows(&qm, q, (uint64_t)h_q * n);
-  if (rc == CRISP_OK) rc = encode_rows(&km, k, (uint64_t)h_kv * n);
+  rc = encode_heads(&qm, q, (uint64_t)n, (uint64_t)h_q);
+  if (rc == CRISP_OK) rc = encode_heads(&km, k, (uint64_t)n, (uint64_t)h_kv);
   if (rc != CRISP_OK) return rc;
   // The array keeps the previous call's contents: clear what the kernels accumulate into.
   if (cudaMemsetAsync(at(w.status), 0, 256, st) != cudaSuccess ||

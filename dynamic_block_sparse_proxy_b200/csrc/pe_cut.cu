@@ -3,7 +3,8 @@
 // pseudocode: gamma_cumsum(pool(Q), pool(K), gamma)).
 //
 // For every head routed to PE:
-//   qbar_kernel     Q_bar[qb] = mean of the block's 128 query rows (fp32), read once from HBM;
+//   qbar_kernel     Q_bar[qb] = mean of the block's query rows (fp32; 128, or fewer in a partial
+//                   last block), read once from HBM;
 //   scores_kernel   logits Q_bar[qb] . K_bar[kb] / sqrt(d) for kb <= qb (128x128 fp32 tiles);
 //   rowsoft_kernel  P[qb, kb] = softmax over kb <= qb, in place, plus the first radix histogram;
 //   cut_select / cut_hist: an exact radix select (11 + 10 + 10 bits of the positive fp32
@@ -32,10 +33,11 @@ __global__ void __launch_bounds__(128) qbar_kernel(const SelectArgs a) {
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  const int rows = min(kB, s.n - qb * kB);  // a partial last block has fewer rows
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const int row = rg + 8 * i;
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(base + (size_t)row * kD));
+    const uint4 u = row < rows ? __ldg(reinterpret_cast<const uint4*>(base + (size_t)row * kD)) : make_uint4(0, 0, 0, 0);
     const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -51,7 +53,7 @@ __global__ void __launch_bounds__(128) qbar_kernel(const SelectArgs a) {
   float v = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) v += red[i][t];
-  a.qbar[((size_t)h * s.nb + qb) * kD + t] = v * (1.f / kB);
+  a.qbar[((size_t)h * s.nb + qb) * kD + t] = v * (1.f / (float)rows);
 }
 
 // -------------------------------------------------------------------------------- logits

@@ -105,10 +105,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       tma_prefetch_desc(&q_map);
       tma_prefetch_desc(&k_map);
       mbar_arrive_expect_tx(&sm.q_full, TILE_BYTES * ntiles);
-      for (int t = 0; t < ntiles; ++t) {
-        const int qrow = (h0 + t) * s.n + s.n - kB;
-        tma_load_2d(&q_map, &sm.q_full, sm.q[t], 0, qrow);
-        tma_load_2d(&q_map, &sm.q_full, sm.q[t] + kB * 64, 64, qrow);
+      for (int t = 0; t < ntiles; ++t) {  // the last 128 queries of each head
+        tma_load_3d(&q_map, &sm.q_full, sm.q[t], 0, s.n - kB, h0 + t);
+        tma_load_3d(&q_map, &sm.q_full, sm.q[t] + kB * 64, 64, s.n - kB, h0 + t);
       }
       int issued = 0;
       for (int j = 0; j < nblk; ++j) {
@@ -117,10 +116,10 @@ __global__ void __launch_bounds__(THREADS, 1)
           fail(sm, a.status);
           break;
         }
-        const int krow = kv * s.n + (kb0 + j) * kB;
+        const int ky = (kb0 + j) * kB;  // rows past n of a partial last block arrive as zeros
         mbar_arrive_expect_tx(&sm.k_full[st], TILE_BYTES);
-        tma_load_2d(&k_map, &sm.k_full[st], sm.k[st], 0, krow);
-        tma_load_2d(&k_map, &sm.k_full[st], sm.k[st] + kB * 64, 64, krow);
+        tma_load_3d(&k_map, &sm.k_full[st], sm.k[st], 0, ky, kv);
+        tma_load_3d(&k_map, &sm.k_full[st], sm.k[st] + kB * 64, 64, ky, kv);
         ++issued;
       }
       // Never leave with copies in flight: wait (bounded) for the last load of each stage.
@@ -170,7 +169,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int grp = warp & 3;
     const int r = grp * 32 + lane;
     const uint32_t lane_off = (uint32_t)(grp * 32) << 16;
+    // With n = 128 (N_b - 1) + t_last, t_last in [1, 128]: row r sits at position n-128+r, a key
+    // at column c of block kb has offset o = n-128+r - 128 kb - c, and the slash block of o is
+    // N_b-2-kb + floor((t_last + r - c) / 128). Columns c <= (t_last + r) mod 128 ("lo") go to the
+    // higher of the two slash blocks a (row, block) meets. When t_last = 128 that column is r.
+    const int t_last = s.n - (s.nb - 1) * kB;
+    const bool ragged = t_last != kB;
+    const int sigma = (t_last + r) & (kB - 1);
     float m = -INFINITY;
+    float rec = 0.f;  // recency-window mass in block N_b-2 (columns >= t_last), ragged n only
     bool ok = true;
     for (int j = 0; j < nblk; ++j) {
       const int b = j & 1;
@@ -186,20 +193,23 @@ __global__ void __launch_bounds__(THREADS, 1)
       // the earlier partial sums rescaled. S stays in TMEM until the block is done.
       uint32_t v[4][32];
       const uint32_t sbase = tmem + t * 256 + b * 128 + lane_off;
-      const bool last = kb0 + j == s.nb - 1;
+      const int kb = kb0 + j;
+      const int lim = s.n - kB + r - kb * kB;  // row r sees columns c <= lim of this block
+      const bool edge = kb >= s.nb - 2;         // only the last two blocks can be cut by lim
+      const bool rec_blk = ragged && s.nb >= 3 && kb == s.nb - 2;
       bool need_max = (m == -INFINITY);
-      float lo = 0.f, hi = 0.f;
+      float lo = 0.f, hi = 0.f, rx = 0.f;
       for (int attempt = 0; attempt < 2; ++attempt) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(sbase + c * 32, v[c]);
         tmem_ld_wait();
-        if (last) {
-          // last key block: row r (position n-B+r) sees keys t <= r only
+        if (edge) {
+          // causal: row r (position n-128+r) sees keys up to its own position only
 #pragma unroll
           for (int c = 0; c < 4; ++c)
 #pragma unroll
             for (int q = 0; q < 32; ++q)
-              if (c * 32 + q > r) v[c][q] = __float_as_uint(-INFINITY);
+              if (c * 32 + q > lim) v[c][q] = __float_as_uint(-INFINITY);
         }
         if (need_max) {
           float mx8[8];
@@ -219,6 +229,7 @@ __global__ void __launch_bounds__(THREADS, 1)
               pv.y *= f;
               sm.part[t][jj][r] = pv;
             }
+            rec *= f;
             m = xm;
           }
         }
@@ -227,6 +238,19 @@ __global__ void __launch_bounds__(THREADS, 1)
         // straddles the diagonal offset lane by lane
         lo = 0.f;
         hi = 0.f;
+        rx = 0.f;
+        if (ragged) {
+          // the split column (t_last + r) mod 128 is not aligned with the warp's lanes
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+              const int col = c * 32 + q;
+              const float e = fast_exp2(fmaf(__uint_as_float(v[c][q]), kScaleLog2, nm));
+              if (col <= sigma) lo += e; else hi += e;
+              if (rec_blk && col >= t_last) rx += e;
+            }
+        } else {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           float s4[4] = {0.f, 0.f, 0.f, 0.f};
@@ -252,6 +276,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             hi += h2[0] + h2[1];
           }
         }
+        }
         const bool redo = !need_max && !(lo + hi <= 18446744073709551616.0f);  // 2^64, or inf / nan
         if (!__any_sync(0xffffffffu, redo)) break;
         need_max = true;
@@ -260,6 +285,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.s_free[t][b]);
       sm.part[t][j][r] = make_float2(lo, hi);
+      if (rec_blk) rec = rx;
     }
     if (ok) {
       const int h = h0 + t;
@@ -272,6 +298,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const size_t ci = ((size_t)h * s.n_chunks + chunk) * kB + r;
       a.chunk_max[ci] = m;
       a.chunk_tot[ci] = tot;
+      if (ragged && s.nb >= 3 && s.nb - 2 >= kb0 && s.nb - 2 < kb0 + nblk) a.rec_extra[(size_t)h * kB + r] = rec;
     }
     __syncwarp();
   } else if (warp >= POOL_WARP) {
@@ -325,7 +352,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
       if (active && rg == 0) {
         float4* dst = reinterpret_cast<float4*>(a.kbar + ((size_t)kv * s.nb + kb0 + j) * kD + cc * 8);
-        const float inv = 1.f / kB;
+        // a partial last block averages the rows it has (the rest arrived as zeros)
+        const float inv = kb0 + j == s.nb - 1 ? 1.f / (float)(s.n - (s.nb - 1) * kB) : 1.f / kB;
         dst[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
         dst[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
       }

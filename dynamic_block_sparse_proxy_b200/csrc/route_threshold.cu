@@ -90,34 +90,49 @@ __global__ void __launch_bounds__(STAT_ROWS * 32) row_stats_kernel(const SelectA
   for (int c = lane; c < s.n_chunks; c += 32) w[c * kB + r] = (float)((double)exp2f(mc[c * kB + r] - M) * inv);
 }
 
-// 2. Block masses, one warp per key block: p_v[kb] = sum_r w*(lo+hi); the lower-offset halves
-//    belong to slash block N_b-1-kb and the upper ones to N_b-2-kb (CRISP §4, both directions).
+// 2. Block masses, one warp per key block: p_v[kb] = sum_r w*(lo+hi). A row r whose split column
+//    is (t_last + r) mod 128 (t_last = n - 128 (N_b-1), 128 when n is a multiple of 128) meets
+//    slash blocks N_b-1-kb (lo) and N_b-2-kb (hi) when t_last + r >= 128, else N_b-2-kb (lo) and
+//    N_b-3-kb (hi) (CRISP §4, both directions). Every slot of ps_lo, ps_hi and ps_x is written
+//    once: by the key block that maps there, or with 0 by the block whose target lies below 0.
 constexpr int MASS_WARPS = 16;
 __global__ void __launch_bounds__(MASS_WARPS * 32) block_mass_kernel(const SelectArgs a) {
   const Shape& s = a.s;
   const int h = blockIdx.y, nb = s.nb;
   const int kb = blockIdx.x * MASS_WARPS + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (kb >= nb) return;
+  const int t_last = s.n - (nb - 1) * kB;
   const float2* p = a.part + ((size_t)h * nb + kb) * kB;
   const float* wc = a.row_w + ((size_t)h * s.n_chunks + kb / kProxyChunk) * kB;
-  double lo = 0.0, hi = 0.0;
+  double loA = 0.0, hiA = 0.0, loB = 0.0, hiB = 0.0;
 #pragma unroll
   for (int i = 0; i < kB / 32; ++i) {
     const int r = lane + 32 * i;
     const float2 v = p[r];
     const double ww = wc[r];
-    lo += (double)v.x * ww;
-    hi += (double)v.y * ww;
+    if (t_last + r >= kB) {
+      loA += (double)v.x * ww;
+      hiA += (double)v.y * ww;
+    } else {
+      loB += (double)v.x * ww;
+      hiB += (double)v.y * ww;
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
-    lo += __shfl_xor_sync(0xffffffffu, lo, o);
-    hi += __shfl_xor_sync(0xffffffffu, hi, o);
+    loA += __shfl_xor_sync(0xffffffffu, loA, o);
+    hiA += __shfl_xor_sync(0xffffffffu, hiA, o);
+    loB += __shfl_xor_sync(0xffffffffu, loB, o);
+    hiB += __shfl_xor_sync(0xffffffffu, hiB, o);
   }
   if (lane == 0) {
-    a.pv[(size_t)h * nb + kb] = lo + hi;
-    a.ps_lo[(size_t)h * nb + nb - 1 - kb] = lo;
-    a.ps_hi[(size_t)h * nb + (nb - 2 - kb >= 0 ? nb - 2 - kb : nb - 1)] = nb - 2 - kb >= 0 ? hi : 0.0;
+    const size_t base = (size_t)h * nb;
+    a.pv[base + kb] = (loA + hiA) + (loB + hiB);
+    a.ps_lo[base + nb - 1 - kb] = loA;
+    if (nb - 2 - kb >= 0) a.ps_hi[base + nb - 2 - kb] = hiA + loB;
+    else a.ps_hi[base + nb - 1] = 0.0;  // kb = N_b-1: the slot no block maps to
+    if (nb - 3 - kb >= 0) a.ps_x[base + nb - 3 - kb] = hiB;
+    else a.ps_x[base + (nb - 3 - kb == -1 ? nb - 2 : nb - 1)] = 0.0;  // kb = N_b-2, N_b-1
   }
 }
 
@@ -294,12 +309,22 @@ __global__ void __launch_bounds__(THREADS) route_threshold_kernel(const SelectAr
   __shared__ int pos_min;
   for (int i = tid; i < nb; i += THREADS) {
     pv[i] = a.pv[(size_t)h * nb + i];
-    ps[i] = a.ps_lo[(size_t)h * nb + i] + (i == nb - 1 ? 0.0 : a.ps_hi[(size_t)h * nb + i]);
+    ps[i] = a.ps_lo[(size_t)h * nb + i] + a.ps_hi[(size_t)h * nb + i] + a.ps_x[(size_t)h * nb + i];
   }
   __syncthreads();
 
-  // C_struct and route
-  const double C = nb >= 2 ? pv[0] + pv[nb - 1] : pv[0];
+  // C_struct: mass on the first 128 keys and the last 128 keys. When n is a multiple of 128 these
+  // are blocks 0 and N_b-1; otherwise the last 128 keys also cover block N_b-2's columns from
+  // t_last on (collected per proxy row by the proxy pass). With N_b = 2 the windows overlap and
+  // their union is every key.
+  double C = nb >= 2 ? pv[0] + pv[nb - 1] : pv[0];
+  const int t_last = s.n - (nb - 1) * kB;
+  if (t_last != kB && nb >= 3) {
+    const float* wr = a.row_w + ((size_t)h * s.n_chunks + (nb - 2) / kProxyChunk) * kB;
+    double x = 0.0;
+    for (int r = tid; r < kB; r += THREADS) x += (double)a.rec_extra[(size_t)h * kB + r] * (double)wr[r];
+    C += block_sum(x, red);
+  }
   double jsd = 0.0;
   int vs;
   if (a.route_rule == 1) {

@@ -9,10 +9,10 @@
  * Conventions shared by every entry point
  *   - Q is bf16 [h_q][n][d], K and V are bf16 [h_kv][n][d], all contiguous, in device memory.
  *     GQA: q-head h reads kv-head h / (h_q / h_kv) (consecutive q-heads share a kv-head).
- *   - Supported shapes: d == 128, block == 128, anchors == 128, h_q a multiple of h_kv, and
- *     n >= 1 for attention alone (crisp_sparse_prefill, crisp_dense_prefill) or n a multiple of
- *     128 with N_b <= 8192 for anything that selects (crisp_select, crisp_prefill,
- *     crisp_select_noalloc). Anything else returns CRISP_ERR_UNSUPPORTED before any launch.
+ *   - Supported shapes: d == 128, block == 128, anchors == 128, h_q a multiple of h_kv, any
+ *     n >= 1 for attention alone (crisp_sparse_prefill, crisp_dense_prefill) and 128 <= n with
+ *     N_b <= 8192 for anything that selects (crisp_select, crisp_prefill, crisp_select_noalloc).
+ *     Anything else returns CRISP_ERR_UNSUPPORTED before any launch.
  *   - N_b = ceil(n / 128) is the number of blocks; when n is not a multiple of 128 the last
  *     query and key blocks are partial (their rows past n do not exist).
  *   - Ownership: the caller allocates every buffer (inputs, outputs, index, workspace); the
@@ -75,7 +75,8 @@ enum {
  * Selection (crisp_select, crisp_prefill, crisp_select_noalloc) keeps per-head block arrays in
  * shared memory and supports N_b <= 8192 (n <= 1,048,576); larger n returns
  * CRISP_ERR_UNSUPPORTED. Attention alone (crisp_sparse_prefill, crisp_dense_prefill) has no
- * such limit.
+ * such limit. When n is not a multiple of 128 the proxy still takes the last 128 queries and
+ * the anchors the first and last 128 keys; a partial last block pools and averages what it has.
  */
 typedef struct {
   int32_t block;

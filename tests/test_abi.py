@@ -48,7 +48,7 @@ def test_workspace_size(L):
     nb = 131072 // 128
     assert big > 8 * 32 * nb * (nb + 1) // 2
     assert big % 256 == 0
-    for bad in [(1, 1, 4096, 64), (1, 1, 4000, 128), (3, 2, 4096, 128), (0, 1, 4096, 128), (1, 1, 0, 128)]:
+    for bad in [(1, 1, 4096, 64), (1, 1, 100, 128), (3, 2, 4096, 128), (0, 1, 4096, 128), (1, 1, 0, 128)]:
         assert L.crisp_workspace_size(*bad, ctypes.byref(p)) == 0
     q = crisp.Params(block=64).c()
     assert L.crisp_workspace_size(1, 1, 4096, 128, ctypes.byref(q)) == 0
@@ -68,7 +68,7 @@ def test_select_rejects_bad_arguments_before_launch(L):
     cases = [
         ((None, fake, 1, 1, 4096, 128, ctypes.byref(p), ctypes.byref(ix), ws, big, None), crisp.STATUS_NAMES[-1]),
         ((fake, fake, 1, 1, 4096, 64, ctypes.byref(p), ctypes.byref(ix), ws, big, None), crisp.STATUS_NAMES[-2]),
-        ((fake, fake, 1, 1, 4000, 128, ctypes.byref(p), ctypes.byref(ix), ws, big, None), crisp.STATUS_NAMES[-2]),
+        ((fake, fake, 1, 1, 100, 128, ctypes.byref(p), ctypes.byref(ix), ws, big, None), crisp.STATUS_NAMES[-2]),
         ((fake, fake, 3, 2, 4096, 128, ctypes.byref(p), ctypes.byref(ix), ws, big, None), crisp.STATUS_NAMES[-2]),
         ((fake, fake, 1, 1, 4096, 128, None, ctypes.byref(ix), ws, big, None), crisp.STATUS_NAMES[-1]),
         ((fake, fake, 1, 1, 4096, 128, ctypes.byref(p), None, ws, big, None), crisp.STATUS_NAMES[-1]),
@@ -89,12 +89,15 @@ def test_select_rejects_bad_arguments_before_launch(L):
 
 
 def test_lengths_not_multiple_of_128(L):
-    # attention runs at any length (workspace sized without params); selection does not
+    # any length sizes a workspace; selection needs n >= 128 (the proxy takes the last 128 queries)
+    # (fake pointers only with arguments refused before any launch)
     p = crisp.Params().c()
     assert L.crisp_workspace_size(2, 1, 1000, 128, None) > 0
-    assert L.crisp_workspace_size(2, 1, 1000, 128, ctypes.byref(p)) == 0
+    assert L.crisp_workspace_size(2, 1, 1000, 128, ctypes.byref(p)) > 0
+    assert L.crisp_workspace_size(2, 1, 100, 128, ctypes.byref(p)) == 0
+    assert L.crisp_workspace_size(2, 1, 100, 128, None) > 0
     ix = _idx()
-    assert L.crisp_select(0x10000, 0x10000, 2, 1, 1000, 128, ctypes.byref(p), ctypes.byref(ix), 0x100000,
+    assert L.crisp_select(0x10000, 0x10000, 2, 1, 100, 128, ctypes.byref(p), ctypes.byref(ix), 0x100000,
                           1 << 40, None) == -2
 
 
@@ -137,3 +140,14 @@ def test_compute_calls_fail_loudly_without_the_library(monkeypatch, tmp_path):
     monkeypatch.setattr(crisp, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError):
         crisp.lib()
+
+
+def test_binding_sizes_the_index_by_ceil_blocks_and_checks_it():
+    assert crisp.n_blocks(300) == 3 and crisp.n_blocks(256) == 2 and crisp.n_blocks(1) == 1
+    # an index the library would overrun is refused before any call (CPU tensors fail the check too)
+    import torch
+    h_q, n = 2, 300
+    small = crisp.Index(torch.zeros(h_q, dtype=torch.int32), torch.zeros(h_q), torch.zeros(h_q, 3, dtype=torch.int32),
+                        torch.zeros(h_q, 3, dtype=torch.int32))
+    with pytest.raises(ValueError):
+        small.check(h_q, n)

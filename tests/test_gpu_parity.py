@@ -320,6 +320,37 @@ def test_flexprefill_full_128k():
                                                        sample_blocks(nb, [0, 2], 1, seed=3), w.h_q // w.h_kv))
 
 
+# ------------------------------------------------------------------ lengths not a multiple of 128
+def _ragged(name, n):
+    """The workload's generator at the next multiple of 128, cut to n tokens."""
+    w = W.WORKLOADS[name].scaled(-(-n // 128) * 128)
+    q, k, v, meta = W.generate(w)
+    cut = lambda t: t[:, :n].contiguous().to(dev())  # noqa: E731
+    return w, cut(q), cut(k), cut(v)
+
+
+@pytest.mark.parametrize("name,n,rules", [("tiny_1h_4k", 300, "crisp"), ("tiny_1h_4k", 200, "crisp"),
+                                          ("llama8b_32k", 4000, "crisp"), ("qwen7b_128k", 3001, "crisp"),
+                                          ("llama8b_32k", 4000, "flexprefill"), ("qwen7b_128k", 2177, "median_floor"),
+                                          ("llama8b_32k", 4095, "crisp"), ("llama8b_32k", 3969, "crisp")])
+def test_ragged_selection_and_attention(name, n, rules):
+    params = {"crisp": crisp.Params(), "flexprefill": crisp.Params.flexprefill(),
+              "median_floor": crisp.Params(floor_rule=1)}[rules]
+    w, q, k, v = _ragged(name, n)
+    nb = -(-n // 128)
+    ws = crisp.workspace(w.h_q, w.h_kv, n, dev())
+    idx = crisp.Index.empty(w.h_q, n, dev(), debug=True)
+    o, lse, idx = crisp.prefill(q, k, v, params, index=idx, ws=ws)
+    crisp.check_status(ws)
+    heads = list(range(w.h_q))
+    sels = PT.oracle_select_heads(q, k, params, heads)
+    PT.compare_selection(idx, sels, nb)
+    G = w.h_q // w.h_kv
+    ah = sorted({0, w.h_q // 2, w.h_q - 1})
+    blocks = [(h, qb) for h in ah for qb in sorted({0, nb // 2, nb - 2, nb - 1}) if qb >= 0]
+    PT.assert_attention_ok(PT.compare_attention_blocks(q, k, v, o, lse, all_lists(idx, ah), blocks, G))
+
+
 # ------------------------------------------------------------------------------ full-size workloads
 def _full(name, sel_heads, attn_per_head, attn_heads=None, seed=0):
     w = W.WORKLOADS[name]
