@@ -23,7 +23,7 @@ STATUS_NAMES = {
 }
 EXPORTED = ["crisp_workspace_size", "crisp_select", "crisp_sparse_prefill", "crisp_prefill",
             "crisp_dense_prefill", "crisp_get_status", "crisp_status_string", "crisp_selftest_timeout",
-            "crisp_select_noalloc"]
+            "crisp_select_noalloc", "crisp_prefill_varlen"]
 
 
 class CrispError(RuntimeError):
@@ -62,12 +62,14 @@ def lib() -> ctypes.CDLL:
         L.crisp_sparse_prefill.argtypes = [vp, vp, vp, i32, i32, i32, i32, I, vp, vp, vp, sz, vp]
         L.crisp_prefill.argtypes = [vp, vp, vp, i32, i32, i32, i32, P, vp, vp, I, vp, sz, vp]
         L.crisp_dense_prefill.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, sz, vp]
+        L.crisp_prefill_varlen.argtypes = [vp, vp, vp, i32, i32, i32, ctypes.POINTER(ctypes.c_int32), i32, i32, P,
+                                           vp, vp, vp, sz, vp]
         L.crisp_get_status.argtypes = [vp, vp]
         L.crisp_status_string.argtypes = [i32]
         L.crisp_status_string.restype = ctypes.c_char_p
         L.crisp_selftest_timeout.argtypes = [vp, sz, ctypes.c_uint64, vp]
         for name in ("crisp_select", "crisp_sparse_prefill", "crisp_prefill", "crisp_dense_prefill",
-                     "crisp_get_status", "crisp_selftest_timeout"):
+                     "crisp_get_status", "crisp_selftest_timeout", "crisp_prefill_varlen"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -246,6 +248,27 @@ def prefill(q, k, v, params: Params | None = None, index: Index | None = None, o
                                o.data_ptr(), lse.data_ptr() if lse is not None else None, ix, ws.data_ptr(),
                                ws.numel(), _stream(q)), "crisp_prefill")
     return o, lse, index
+
+
+def prefill_varlen(q, k, v, cu_seqlens, params: Params | None = None, o=None, lse=None, ws=None,
+                   want_lse: bool = True):
+    """crisp_prefill over independent sequences packed along the tokens (crisp_prefill_varlen).
+    cu_seqlens: host sequence of n_seqs+1 offsets into the token axis. Returns (o, lse)."""
+    h_q, h_kv, total, d = _qkv_shape(q, k, v)
+    cu = [int(x) for x in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
+    params = params or Params()
+    longest = max((b - a for a, b in zip(cu[:-1], cu[1:])), default=0)
+    ws = ws if ws is not None else workspace(h_q, h_kv, max(longest, 1), q.device, d)
+    o = o if o is not None else torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(h_q, total, device=q.device, dtype=torch.float32)
+    _check_out(q, o, lse)
+    arr = (ctypes.c_int32 * len(cu))(*cu)
+    p = params.c()
+    _check(lib().crisp_prefill_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), h_q, h_kv, total, arr, len(cu) - 1,
+                                      d, ctypes.byref(p), o.data_ptr(), lse.data_ptr() if lse is not None else None,
+                                      ws.data_ptr(), ws.numel(), _stream(q)), "crisp_prefill_varlen")
+    return o, lse
 
 
 def dense_prefill(q, k, v, o=None, lse=None, ws=None, want_lse: bool = True):

@@ -25,13 +25,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 3D bf16 view [heads][n][128] with 64x128x1 boxes: a head's rows past n read as zeros, so a
-// partial last block never sees the next head's rows.
-int make_map3(CUtensorMap* m, const void* base, uint64_t n, uint64_t heads) {
+// 3D bf16 view [heads][n][128] (heads `ld` rows apart) with 64x128x1 boxes: a head's rows past n
+// read as zeros, so a partial last block never sees the next head's (or sequence's) rows.
+int make_map3(CUtensorMap* m, const void* base, uint64_t n, uint64_t heads, uint64_t ld) {
   auto fn = encode_fn();
   if (fn == nullptr) return CRISP_ERR_CUDA;
   cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)n, (cuuint64_t)heads};
-  cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)kD * 2 * n};
+  cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)kD * 2 * ld};
   cuuint32_t box[3] = {64, (cuuint32_t)kB, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
@@ -53,6 +53,7 @@ int check_shape(int h_q, int h_kv, int n, int d, Shape* s) {
   s->h_q = h_q;
   s->h_kv = h_kv;
   s->n = n;
+  s->ld = n;
   s->nb = (int)nb;
   s->G = h_q / h_kv;
   s->n_chunks = (int)((nb + kProxyChunk - 1) / kProxyChunk);
@@ -133,8 +134,8 @@ int run_select(const void* q, const void* k, const Shape& s, const crisp_params*
   a.debug = out.debug;
 
   CUtensorMap qm, km;
-  int rc = make_map3(&qm, q, (uint64_t)s.n, (uint64_t)s.h_q);
-  if (rc == CRISP_OK) rc = make_map3(&km, k, (uint64_t)s.n, (uint64_t)s.h_kv);
+  int rc = make_map3(&qm, q, (uint64_t)s.n, (uint64_t)s.h_q, (uint64_t)s.ld);
+  if (rc == CRISP_OK) rc = make_map3(&km, k, (uint64_t)s.n, (uint64_t)s.h_kv, (uint64_t)s.ld);
   if (rc != CRISP_OK) return rc;
 
   // The radix histograms accumulate with atomics: start from zero.
@@ -165,9 +166,9 @@ int run_attention(const void* q, const void* k, const void* v, const Shape& s, c
   a.trace = at<unsigned long long>(ws, w.trace);
   a.scale_log2 = 0.12751743074380045f;  // log2(e) / sqrt(128)
   CUtensorMap qm, km, vm;
-  int rc = make_map3(&qm, q, (uint64_t)s.n, (uint64_t)s.h_q);
-  if (rc == CRISP_OK) rc = make_map3(&km, k, (uint64_t)s.n, (uint64_t)s.h_kv);
-  if (rc == CRISP_OK) rc = make_map3(&vm, v, (uint64_t)s.n, (uint64_t)s.h_kv);
+  int rc = make_map3(&qm, q, (uint64_t)s.n, (uint64_t)s.h_q, (uint64_t)s.ld);
+  if (rc == CRISP_OK) rc = make_map3(&km, k, (uint64_t)s.n, (uint64_t)s.h_kv, (uint64_t)s.ld);
+  if (rc == CRISP_OK) rc = make_map3(&vm, v, (uint64_t)s.n, (uint64_t)s.h_kv, (uint64_t)s.ld);
   if (rc != CRISP_OK) return rc;
   return launch_sparse_attn(qm, km, vm, a, st) == cudaSuccess ? CRISP_OK : CRISP_ERR_CUDA;
 }
@@ -260,6 +261,58 @@ int crisp_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv
   rc = run_select(q, k, s, params, idx, ws, st);
   if (rc != CRISP_OK) return rc;
   return run_attention(q, k, v, s, idx.row_ptr, idx.cols, idx.route, 0, o, lse, ws, st);
+}
+
+int crisp_prefill_varlen(const void* q, const void* k, const void* v, int h_q, int h_kv, int total,
+                         const int32_t* cu_seqlens, int n_seqs, int d, const crisp_params* params, void* o,
+                         float* lse, void* ws, size_t ws_bytes, void* stream) {
+  // every check comes before the first launch
+  Shape whole;
+  int rc = check_shape(h_q, h_kv, total, d, &whole);
+  if (rc == CRISP_OK) rc = check_params(params);
+  if (rc == CRISP_OK && (!tensors_ok(q, k, v) || v == nullptr || o == nullptr || !aligned(o, 16)))
+    rc = CRISP_ERR_INVALID_ARG;
+  if (rc == CRISP_OK && (cu_seqlens == nullptr || n_seqs <= 0 || cu_seqlens[0] != 0 || cu_seqlens[n_seqs] != total))
+    rc = CRISP_ERR_INVALID_ARG;
+  int longest = 0;
+  for (int i = 0; rc == CRISP_OK && i < n_seqs; ++i) {
+    const int len = cu_seqlens[i + 1] - cu_seqlens[i];
+    if (len < 0) rc = CRISP_ERR_INVALID_ARG;
+    else if (len > 0 && len < kB) rc = CRISP_ERR_UNSUPPORTED;  // selection takes the last 128 queries
+    longest = len > longest ? len : longest;
+  }
+  Shape big;
+  if (rc == CRISP_OK) rc = longest > 0 ? check_shape(h_q, h_kv, longest, d, &big) : CRISP_ERR_INVALID_ARG;
+  if (rc == CRISP_OK && big.nb > kMaxSelectBlocks) rc = CRISP_ERR_UNSUPPORTED;
+  if (rc == CRISP_OK) rc = check_ws(ws, ws_bytes, big);
+  if (rc != CRISP_OK) return rc;
+  // One sequence after another on the stream, each on the same workspace (its index included);
+  // a sequence's tensors start at its first token and keep the batch's per-head stride.
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int i = 0; i < n_seqs; ++i) {
+    const int beg = cu_seqlens[i], len = cu_seqlens[i + 1] - beg;
+    if (len == 0) continue;
+    Shape s;
+    check_shape(h_q, h_kv, len, d, &s);
+    s.ld = total;
+    const Workspace w = workspace_layout(s);
+    crisp_index idx;
+    idx.route = at<int32_t>(ws, w.idx_route);
+    idx.c_struct = at<float>(ws, w.idx_c);
+    idx.row_ptr = at<int32_t>(ws, w.idx_row_ptr);
+    idx.cols = at<int32_t>(ws, w.idx_cols);
+    idx.debug = nullptr;
+    const size_t off = (size_t)beg * kD;
+    const auto* qs = static_cast<const __nv_bfloat16*>(q) + off;
+    const auto* ks = static_cast<const __nv_bfloat16*>(k) + off;
+    const auto* vs = static_cast<const __nv_bfloat16*>(v) + off;
+    auto* os = static_cast<__nv_bfloat16*>(o) + off;
+    rc = run_select(qs, ks, s, params, idx, ws, st);
+    if (rc == CRISP_OK) rc = run_attention(qs, ks, vs, s, idx.row_ptr, idx.cols, idx.route, 0, os,
+                                           lse != nullptr ? lse + beg : nullptr, ws, st);
+    if (rc != CRISP_OK) return rc;
+  }
+  return CRISP_OK;
 }
 
 int crisp_dense_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv, int n, int d, void* o,

@@ -21,6 +21,7 @@ constexpr double kMassUnit = 1099511627776.0;  // 2^40: fixed-point scale of his
 
 struct Shape {
   int h_q, h_kv, n, nb, G, n_chunks;
+  int ld;  // rows between consecutive heads in Q, K, V, O and LSE (n, or the packed batch length)
   long long cap;  // per-head capacity of the column array: nb*(nb+1)/2
 };
 

@@ -93,6 +93,7 @@ extern "C" int crisp_select_noalloc(const void* q, const void* k, int h_q, int h
   s.h_q = h_q;
   s.h_kv = h_kv;
   s.n = n;
+  s.ld = n;
   s.nb = (int)nb;
   s.G = h_q / h_kv;
   s.n_chunks = (int)((nb + kProxyChunk - 1) / kProxyChunk);

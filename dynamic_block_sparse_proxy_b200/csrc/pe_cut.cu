@@ -29,7 +29,7 @@ __global__ void __launch_bounds__(128) qbar_kernel(const SelectArgs a) {
   if (!is_pe(a, h)) return;
   const Shape& s = a.s;
   const int t = threadIdx.x, c16 = t & 15, rg = t >> 4;
-  const __nv_bfloat16* base = a.q + ((size_t)h * s.n + (size_t)qb * kB) * kD + c16 * 8;
+  const __nv_bfloat16* base = a.q + ((size_t)h * s.ld + (size_t)qb * kB) * kD + c16 * 8;
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;

@@ -160,7 +160,7 @@ __device__ double jsd_statistic(const SelectArgs& a, int h, const double* pv, do
   // mean of the last 128 query rows; thread t sums column t%128 over rows t/128, t/128+4, ...
   {
     const int col = tid & (kD - 1), rg = tid >> 7;
-    const __nv_bfloat16* qrow = a.q + ((size_t)h * s.n + (size_t)(s.n - kB)) * kD + col;
+    const __nv_bfloat16* qrow = a.q + ((size_t)h * s.ld + (size_t)(s.n - kB)) * kD + col;
     float acc = 0.f;
     for (int r = rg; r < kB; r += THREADS / kD) acc += __bfloat162float(qrow[(size_t)r * kD]);
     qpart[rg][col] = acc;

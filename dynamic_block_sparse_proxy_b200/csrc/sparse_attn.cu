@@ -504,7 +504,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       } else {
         tc_fence_after();
         const float inv = 1.f / l;
-        const size_t row = (size_t)my_h * s.n + (size_t)my_qb * kB + r;
+        const size_t row = (size_t)my_h * s.ld + (size_t)my_qb * kB + r;
         const bool real = my_qb * kB + r < s.n;  // rows past n of a partial last block are not stored
         uint4* dst = reinterpret_cast<uint4*>(a.o + row * kD);
 #pragma unroll

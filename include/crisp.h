@@ -148,6 +148,24 @@ int crisp_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv
                   void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * crisp_prefill over a batch of independent sequences packed along the token axis (a batch has
+ * no counterpart on the pages, which treat one sequence; each sequence here is selected and
+ * attended exactly as crisp_prefill would treat it alone).
+ *   q: bf16 [h_q][total][d], k and v: bf16 [h_kv][total][d]; o: bf16 [h_q][total][d];
+ *   lse: fp32 [h_q][total] or NULL. Sequence i is tokens cu_seqlens[i] .. cu_seqlens[i+1]-1 of
+ *   every head.
+ *   cu_seqlens: HOST int32 [n_seqs+1], cu_seqlens[0] = 0, non-decreasing, cu_seqlens[n_seqs] =
+ *   total; every non-empty sequence needs >= 128 tokens (else CRISP_ERR_UNSUPPORTED); empty ones
+ *   are skipped.
+ *   ws: sized by crisp_workspace_size for the longest sequence; the sequences run one after
+ *   another on `stream` and reuse it (their index sets live there and are not returned).
+ * All checks happen before the first launch; a refused call launches nothing.
+ */
+int crisp_prefill_varlen(const void* q, const void* k, const void* v, int h_q, int h_kv, int total,
+                         const int32_t* cu_seqlens, int n_seqs, int d, const crisp_params* params,
+                         void* o, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Dense causal attention with the same kernel (every block <= qb selected): the reference
  * point for the sparse-versus-dense speed ratio. Same buffers as crisp_sparse_prefill.
  */

@@ -151,3 +151,24 @@ def test_binding_sizes_the_index_by_ceil_blocks_and_checks_it():
                         torch.zeros(h_q, 3, dtype=torch.int32))
     with pytest.raises(ValueError):
         small.check(h_q, n)
+
+
+def test_varlen_refuses_bad_batches_before_launch(L):
+    # (fake pointers only with arguments refused before any launch)
+    p = crisp.Params().c()
+    fake, ws, big = 0x10000, 0x100000, 1 << 40
+    I32 = ctypes.c_int32
+
+    def call(cu, total, ws_bytes=big):
+        arr = (I32 * len(cu))(*cu)
+        return L.crisp_prefill_varlen(fake, fake, fake, 2, 1, total, arr, len(cu) - 1, 128, ctypes.byref(p), fake,
+                                      None, ws, ws_bytes, None)
+
+    assert L.crisp_prefill_varlen(fake, fake, fake, 2, 1, 512, None, 2, 128, ctypes.byref(p), fake, None, ws, big,
+                                  None) == -1
+    assert call([1, 256, 512], 512) == -1          # does not start at 0
+    assert call([0, 256, 500], 512) == -1          # does not end at total
+    assert call([0, 300, 256, 512], 512) == -1     # decreasing
+    assert call([0, 50, 512], 512) == -2           # a sequence shorter than 128 tokens
+    assert call([0, 256, 512], 512, ws_bytes=100) == -3
+    assert call([0, 0, 0], 0) == -1                # nothing to do (total = 0)

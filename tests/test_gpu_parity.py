@@ -351,6 +351,42 @@ def test_ragged_selection_and_attention(name, n, rules):
     PT.assert_attention_ok(PT.compare_attention_blocks(q, k, v, o, lse, all_lists(idx, ah), blocks, G))
 
 
+def test_varlen_batch_equals_single_sequences():
+    """A packed batch gives, for every sequence, exactly what crisp_prefill gives for that sequence
+    alone (same kernels, same inputs), and the oracle agrees on sampled blocks."""
+    import dataclasses
+    lens = [300, 1024, 128, 0, 2177]
+    seqs = []
+    for i, n in enumerate(lens):
+        if n == 0:
+            seqs.append(None)
+            continue
+        w = dataclasses.replace(W.WORKLOADS["llama8b_32k"].scaled(-(-n // 128) * 128), seed=100 + i)
+        q, k, v, _ = W.generate(w)
+        seqs.append(tuple(t[:, :n].contiguous() for t in (q, k, v)))
+    parts = [s for s in seqs if s is not None]
+    q, k, v = (torch.cat([s[j] for s in parts], dim=1).to(dev()) for j in range(3))
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    params = crisp.Params()
+    o, lse = crisp.prefill_varlen(q, k, v, cu, params)
+    torch.cuda.synchronize()
+    G = q.shape[0] // k.shape[0]
+    for i, n in enumerate(lens):
+        if n == 0:
+            continue
+        qs, ks, vs = (t.to(dev()) for t in seqs[i])
+        ws = crisp.workspace(qs.shape[0], ks.shape[0], n, dev())
+        os_, ls_, idx = crisp.prefill(qs, ks, vs, params, ws=ws)
+        crisp.check_status(ws)
+        b, e = int(cu[i]), int(cu[i + 1])
+        assert torch.equal(o[:, b:e], os_), i
+        assert torch.equal(lse[:, b:e], ls_), i
+        nb = -(-n // 128)
+        heads = [0, 17]
+        PT.assert_attention_ok(PT.compare_attention_blocks(qs, ks, vs, os_, ls_, all_lists(idx, heads),
+                                                           [(h, qb) for h in heads for qb in {0, nb - 1}], G))
+
+
 # ------------------------------------------------------------------------------ full-size workloads
 def _full(name, sel_heads, attn_per_head, attn_heads=None, seed=0):
     w = W.WORKLOADS[name]
