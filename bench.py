@@ -132,8 +132,8 @@ def select_bytes(w, n_pe_heads: int, total_pairs: int) -> float:
 # workload, from a one-pass ncu capture of this command's own launch. The figure belongs to the
 # kernel source it was taken on; for any other source or workload the bench reports null.
 ATTN_TRAFFIC = {"workload": "llama8b_128k",
-                "source_sha256": "7054caa5815700d80cac3ad12fe8f9f681f6e55e29d62e7fb58b6b6c14a9577f",
-                "bytes": 2.69e9 + 1.06e9}
+                "source_sha256": "7d0a430321f4f231d5978bce192dbc519320892784022e99096184bcd0f21f1a",
+                "bytes": 2.66e9 + 1.06e9}
 
 
 def attn_traffic(w):
