@@ -19,6 +19,7 @@ import json
 import os
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -77,7 +78,9 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.idx = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        # raw samples go to the temp directory (or CRISP_CLOCKS_DIR); the JSON line carries the summary
+        self.path = os.path.join(os.environ.get("CRISP_CLOCKS_DIR", tempfile.gettempdir()),
+                                 f"crisp_clocks_rank{gpu_index}_{os.getpid()}.csv")
 
     def start(self):
         try:
