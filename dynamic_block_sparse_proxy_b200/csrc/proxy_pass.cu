@@ -52,6 +52,9 @@ __device__ __forceinline__ void fail(ProxySmem& sm, int* status) {
   *reinterpret_cast<volatile int*>(&sm.abort) = 1;
 }
 
+// RAGGED: n is not a multiple of 128 (separate instance, so the common case keeps the lane-aligned
+// split with no extra work in its exponential loop).
+template <bool RAGGED>
 __global__ void __launch_bounds__(THREADS, 1)
     proxy_pass_kernel(const __grid_constant__ CUtensorMap q_map,
                       const __grid_constant__ CUtensorMap k_map, const SelectArgs a) {
@@ -174,7 +177,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // N_b-2-kb + floor((t_last + r - c) / 128). Columns c <= (t_last + r) mod 128 ("lo") go to the
     // higher of the two slash blocks a (row, block) meets. When t_last = 128 that column is r.
     const int t_last = s.n - (s.nb - 1) * kB;
-    const bool ragged = t_last != kB;
+    constexpr bool ragged = RAGGED;
     const int sigma = (t_last + r) & (kB - 1);
     float m = -INFINITY;
     float rec = 0.f;  // recency-window mass in block N_b-2 (columns >= t_last), ragged n only
@@ -195,7 +198,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t sbase = tmem + t * 256 + b * 128 + lane_off;
       const int kb = kb0 + j;
       const int lim = s.n - kB + r - kb * kB;  // row r sees columns c <= lim of this block
-      const bool edge = kb >= s.nb - 2;         // only the last two blocks can be cut by lim
+      const bool edge = RAGGED ? kb >= s.nb - 2 : kb == s.nb - 1;  // blocks lim can cut
       const bool rec_blk = ragged && s.nb >= 3 && kb == s.nb - 2;
       bool need_max = (m == -INFINITY);
       float lo = 0.f, hi = 0.f, rx = 0.f;
@@ -239,7 +242,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         lo = 0.f;
         hi = 0.f;
         rx = 0.f;
-        if (ragged) {
+        if constexpr (RAGGED) {
           // the split column (t_last + r) mod 128 is not aligned with the warp's lanes
 #pragma unroll
           for (int c = 0; c < 4; ++c)
@@ -377,12 +380,13 @@ __global__ void __launch_bounds__(THREADS, 1)
 cudaError_t launch_proxy_pass(const CUtensorMap& q_map, const CUtensorMap& k_map, const SelectArgs& a,
                               cudaStream_t st) {
   const size_t smem = sizeof(ProxySmem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(proxy_pass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  const bool ragged = a.s.n % kB != 0;
+  auto kernel = ragged ? proxy_pass_kernel<true> : proxy_pass_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int n_pairs = a.s.h_kv * ((a.s.G + 1) / 2);
   dim3 grid(n_pairs * a.s.n_chunks);
-  proxy_pass_kernel<<<grid, THREADS, smem, st>>>(q_map, k_map, a);
+  kernel<<<grid, THREADS, smem, st>>>(q_map, k_map, a);
   return cudaGetLastError();
 }
 
