@@ -126,6 +126,7 @@ int run_select(const void* q, const void* k, const Shape& s, const crisp_params*
   a.cnt = at<int>(ws, w.cnt);
   a.eqcnt = at<int>(ws, w.eqcnt);
   a.eqbase = at<int>(ws, w.eqbase);
+  a.selmask = at<uint32_t>(ws, w.selmask);
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.route = out.route;
   a.c_struct = out.c_struct;

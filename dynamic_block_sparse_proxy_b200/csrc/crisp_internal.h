@@ -40,10 +40,13 @@ struct CutState {
 struct Workspace {
   size_t status, trace, part, chunk_max, chunk_tot, row_w, pv, ps_lo, ps_hi, ps_x, rec_extra, kbar, qbar, pbuf,
       hist_cnt, hist_mass, cut,
-      keep_v, keep_s, cnt, eqcnt, eqbase, idx_route, idx_c, idx_row_ptr, idx_cols, total;
+      keep_v, keep_s, cnt, eqcnt, eqbase, selmask, idx_route, idx_c, idx_row_ptr, idx_cols, total;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// 32-bit words of one row's selection bitmask: blocks are decided 128 at a time, 32 per word.
+inline __host__ __device__ int sel_mask_words(int nb) { return 4 * ((nb + 127) / 128); }
 
 inline Workspace workspace_layout(const Shape& s) {
   Workspace w{};
@@ -76,6 +79,7 @@ inline Workspace workspace_layout(const Shape& s) {
   w.cnt = take(hq * nb * 4);
   w.eqcnt = take(hq * nb * 4);
   w.eqbase = take(hq * (nb + 1) * 4);
+  w.selmask = take(hq * nb * (size_t)sel_mask_words((int)nb) * 4);
   w.idx_route = take(hq * 4);
   w.idx_c = take(hq * 4);
   w.idx_row_ptr = take(hq * (nb + 1) * 4);
@@ -115,6 +119,7 @@ struct SelectArgs {
   int* cnt;
   int* eqcnt;
   int* eqbase;
+  uint32_t* selmask;  // per (head, query block): bit kb set iff key block kb is selected
   const __nv_bfloat16* q;
   int32_t* route;
   float* c_struct;

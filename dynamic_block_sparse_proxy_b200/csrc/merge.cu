@@ -92,7 +92,7 @@ __device__ __forceinline__ void stage_flags(const SelectArgs& a, int h, uint8_t*
 
 template <typename Emit>
 __device__ __forceinline__ int walk_row(const SelectArgs& a, int h, int qb, long long erank, const uint8_t* skv,
-                                        const uint8_t* sks, Emit emit) {
+                                        const uint8_t* sks, Emit emit, uint32_t* mrow = nullptr) {
   RowCtx c = make_ctx(a, h, qb);
   if (a.s.nb <= kMaxStagedBlocks) {
     c.kv = skv;
@@ -132,6 +132,7 @@ __device__ __forceinline__ int walk_row(const SelectArgs& a, int h, int qb, long
       }
       const unsigned sb = __ballot_sync(0xffffffffu, sel);
       if (sel) emit(kb, count + __popc(sb & below));
+      if (mrow != nullptr && lane == 0) mrow[base / 32 + u] = sb;  // blocks base+32u .. +31
       count += __popc(sb);
     }
   }
@@ -162,20 +163,38 @@ __global__ void __launch_bounds__(ROWS * 32) merge_count_kernel(const SelectArgs
   stage_flags(a, h, skv, sks);
   if (qb >= a.s.nb) return;
   const long long erank = a.eqbase[(size_t)h * (a.s.nb + 1) + qb];
-  const int n = walk_row(a, h, qb, erank, skv, sks, [](int, int) {});
+  uint32_t* mrow = a.selmask + ((size_t)h * a.s.nb + qb) * sel_mask_words(a.s.nb);
+  const int n = walk_row(a, h, qb, erank, skv, sks, [](int, int) {}, mrow);
   if ((threadIdx.x & 31) == 0) a.cnt[(size_t)h * a.s.nb + qb] = n;
 }
 
-// Pass 3: compaction into the CSR column array.
+// Pass 3: compaction into the CSR column array, from the bitmask the count pass left: one warp per
+// row, 32 words per round, an exclusive scan of their popcounts gives each lane its positions.
 __global__ void __launch_bounds__(ROWS * 32) merge_write_kernel(const SelectArgs a) {
   const int qb = blockIdx.x * ROWS + (threadIdx.x >> 5), h = blockIdx.y;
-  const int nb = a.s.nb;
-  __shared__ uint8_t skv[kMaxStagedBlocks], sks[kMaxStagedBlocks];
-  stage_flags(a, h, skv, sks);
+  const int nb = a.s.nb, lane = threadIdx.x & 31;
   if (qb >= nb) return;
-  const long long erank = a.eqbase[(size_t)h * (nb + 1) + qb];
+  const uint32_t* m = a.selmask + ((size_t)h * nb + qb) * sel_mask_words(nb);
   int32_t* out = a.cols + (size_t)h * a.s.cap + a.row_ptr[(size_t)h * (nb + 1) + qb];
-  walk_row(a, h, qb, erank, skv, sks, [out](int kb, int pos) { out[pos] = kb; });
+  const int nw = qb / 32 + 1;  // words that hold blocks 0..qb
+  int pos = 0;
+  for (int w0 = 0; w0 < nw; w0 += 32) {
+    const int w = w0 + lane;
+    uint32_t bits = w < nw ? m[w] : 0u;
+    const int c = __popc(bits);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int p = pos + incl - c;
+    while (bits) {
+      out[p++] = w * 32 + (__ffs(bits) - 1);
+      bits &= bits - 1;
+    }
+    pos += __shfl_sync(0xffffffffu, incl, 31);
+  }
 }
 
 // One CTA per head: exclusive scan of in[h][0..nb) into out[h][0..nb] (out[nb] = total).

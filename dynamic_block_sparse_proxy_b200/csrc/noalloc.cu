@@ -139,6 +139,7 @@ extern "C" int crisp_select_noalloc(const void* q, const void* k, int h_q, int h
   a.cnt = reinterpret_cast<int*>(at(w.cnt));
   a.eqcnt = reinterpret_cast<int*>(at(w.eqcnt));
   a.eqbase = reinterpret_cast<int*>(at(w.eqbase));
+  a.selmask = reinterpret_cast<uint32_t*>(at(w.selmask));
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.route = out->route;
   a.c_struct = out->c_struct;
