@@ -169,31 +169,25 @@ __global__ void __launch_bounds__(ROWS * 32) merge_count_kernel(const SelectArgs
 }
 
 // Pass 3: compaction into the CSR column array, from the bitmask the count pass left: one warp per
-// row, 32 words per round, an exclusive scan of their popcounts gives each lane its positions.
+// row takes one word at a time, lane j writing block 32w+j if its bit is set, so the stores of a
+// word are contiguous.
 __global__ void __launch_bounds__(ROWS * 32) merge_write_kernel(const SelectArgs a) {
   const int qb = blockIdx.x * ROWS + (threadIdx.x >> 5), h = blockIdx.y;
   const int nb = a.s.nb, lane = threadIdx.x & 31;
   if (qb >= nb) return;
   const uint32_t* m = a.selmask + ((size_t)h * nb + qb) * sel_mask_words(nb);
   int32_t* out = a.cols + (size_t)h * a.s.cap + a.row_ptr[(size_t)h * (nb + 1) + qb];
+  const unsigned below = (1u << lane) - 1u;
   const int nw = qb / 32 + 1;  // words that hold blocks 0..qb
   int pos = 0;
   for (int w0 = 0; w0 < nw; w0 += 32) {
-    const int w = w0 + lane;
-    uint32_t bits = w < nw ? m[w] : 0u;
-    const int c = __popc(bits);
-    int incl = c;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
+    const uint32_t mine = w0 + lane < nw ? m[w0 + lane] : 0u;  // one load per lane, then shared
+    const int cnt = min(32, nw - w0);
+    for (int i = 0; i < cnt; ++i) {
+      const uint32_t bits = __shfl_sync(0xffffffffu, mine, i);
+      if ((bits >> lane) & 1u) out[pos + __popc(bits & below)] = (w0 + i) * 32 + lane;
+      pos += __popc(bits);
     }
-    int p = pos + incl - c;
-    while (bits) {
-      out[p++] = w * 32 + (__ffs(bits) - 1);
-      bits &= bits - 1;
-    }
-    pos += __shfl_sync(0xffffffffu, incl, 31);
   }
 }
 
