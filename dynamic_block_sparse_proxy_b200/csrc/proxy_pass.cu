@@ -8,8 +8,8 @@
 //   warp 9      one thread issues S_t = Q_t K_blk^T (128x128x128, bf16 -> fp32) into a
 //               double-buffered TMEM tile per head;
 //   warps 0-7   softmax, one warpgroup per head, one proxy row per thread: read the S row with
-//               one TMEM round trip, mask the last key block (key j visible to row r iff
-//               j <= n-B+r), and accumulate exp2(x - m) against a lagging row reference m (set
+//               one TMEM round trip, mask the keys the causal limit cuts (key j visible to row r
+//               iff j <= n-B+r), and accumulate exp2(x - m) against a lagging row reference m (set
 //               by the chunk's first block, moved only when a block's sum would leave
 //               [0, 2^64]) into two sums per key block: keys at or below the row's diagonal
 //               offset (t <= r) and above it (t > r);
@@ -17,7 +17,10 @@
 //               CTAs of one group share the 16 column chunks between them.
 // A key at offset t of block kb seen by proxy row r lies on diagonal offset (N_b-1-kb)*B + (r-t),
 // so the first sum belongs to slash block N_b-1-kb and the second to N_b-2-kb; their total is
-// the block's vertical mass. The per-row normalisation happens in the routing kernels.
+// the block's vertical mass. When n is not a multiple of 128 (t_last keys in the last block) the
+// split column is (t_last + r) mod 128, rows with t_last + r < 128 land one slash block lower, and
+// each row also sums block N_b-2's part of the last-128-keys window for C_struct; that case runs in
+// its own kernel instance. The per-row normalisation happens in the routing kernels.
 #include "crisp_internal.h"
 #include "sm100.cuh"
 
