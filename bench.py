@@ -366,7 +366,14 @@ def oracle_baseline(w, q, k, v, idx, budget_s: float, seed: int = 0, params=None
         O.attention_block(f64(q[h, qb * 128:(qb + 1) * 128]), kk, vv, lists[qb], qb)
         t_attn += time.perf_counter() - t0
         pairs_done += len(lists[qb])
-    total_pairs = int(idx.row_ptr[:, nb].sum().item()) if idx is not None else pairs_done
+    if idx is not None:
+        total_pairs = int(idx.row_ptr[:, nb].sum().item())
+    else:
+        # no GPU index (the oracle arm alone): the layer's selected pairs from the oracle's own
+        # lists of the timed heads, each standing for the heads of its kind
+        per = {h: sum(len(x) for x in sel[h]["lists"]) for h in heads}
+        total_pairs = per[vs_head if vs_head is not None else pe_head] * n_vs + \
+            per[pe_head if pe_head is not None else vs_head] * n_pe
     attn_layer = t_attn / max(pairs_done, 1) * total_pairs
     layer_s = sel_layer + attn_layer
     try:
