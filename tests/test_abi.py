@@ -172,3 +172,30 @@ def test_varlen_refuses_bad_batches_before_launch(L):
     assert call([0, 50, 512], 512) == -2           # a sequence shorter than 128 tokens
     assert call([0, 256, 512], 512, ws_bytes=100) == -3
     assert call([0, 0, 0], 0) == -1                # nothing to do (total = 0)
+
+
+def test_params_pack_into_the_c_struct():
+    p = crisp.Params.flexprefill(gamma=0.9, tau_jsd=0.2).c()
+    assert (p.block, p.anchors, p.route_rule, p.vs_rule, p.floor_rule) == (128, 128, 1, 1, 0)
+    assert abs(p.gamma - 0.9) < 1e-7 and abs(p.tau_jsd - 0.2) < 1e-7
+    assert ctypes.sizeof(crisp._Params) == 40  # 10 four-byte fields, as in include/crisp.h
+    q = crisp.Params(floor_rule=1, min_blocks=8).c()
+    assert (q.floor_rule, q.min_blocks, q.route_rule) == (1, 8, 0)
+
+
+def test_binding_refuses_outputs_of_the_wrong_shape_before_calling():
+    import torch
+    q = torch.zeros(2, 256, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        crisp._check_out(q, torch.zeros(2, 256, 128, dtype=torch.float32), None)     # dtype
+    with pytest.raises(ValueError):
+        crisp._check_out(q, torch.zeros(2, 256, 128, dtype=torch.bfloat16), None)    # not on the GPU
+    with pytest.raises(ValueError):
+        crisp._qkv_shape(q, q)                                                       # CPU tensors
+
+
+def test_workspace_grows_with_length_including_partial_blocks(L):
+    sizes = [L.crisp_workspace_size(4, 2, n, 128, None) for n in (1, 127, 128, 129, 1000, 1024, 1025)]
+    assert all(s > 0 and s % 256 == 0 for s in sizes)
+    assert sizes == sorted(sizes)
+    assert sizes[2] == L.crisp_workspace_size(4, 2, 128, 128, None) and sizes[3] > sizes[2]
