@@ -206,6 +206,10 @@ def test_sink_only_collapse():
     assert sorted(kept.tolist()) == g["gamma_keeps"]
     assert abs(O.noise_floor(p) - g["mu"]) < 1e-15
     assert O.keep_blocks(p, 1.0) == g["alpha_mu_keeps"]
+    # FlexPrefill's per-direction rule is the same gamma cut on one direction: it keeps only the
+    # sink anchor, so no inner block survives
+    inner, cut = O.gamma_keep_direction(p, g["gamma"])
+    assert inner == [j for j in g["gamma_keeps"] if 0 < j < nb - 1] == [] and cut == g["p0"]
 
 
 def test_o_n_noise_growth():
@@ -219,6 +223,8 @@ def test_o_n_noise_growth():
         kept, _, _ = O.gamma_cut(p, g["gamma"], 1.0)
         non_anchor = [j for j in kept.tolist() if 0 < j < nb - 1]
         assert len(non_anchor) == want_gamma
+        # the same count through FlexPrefill's per-direction rule
+        assert len(O.gamma_keep_direction(p, g["gamma"])[0]) == want_gamma
         keep = O.keep_blocks(p, 1.0)
         assert len(keep) == want_mu and keep == sorted(sig)
 
