@@ -459,3 +459,83 @@ def test_block_mean_of_a_partial_block():
     assert m.shape == (3, 2)
     np.testing.assert_allclose(m[2], x[256:300].mean(axis=0))   # 44 rows, not 128
     np.testing.assert_allclose(O.pool_blocks(np.ones(300), 128), [128, 128, 44])
+
+
+# ---------------------------------------------------------------- pooled scores, non-uniform rows
+def _pooled_case():
+    with open(os.path.join(os.path.dirname(__file__), "golden", "pooled_scores_case.json")) as f:
+        g = json.load(f)
+    named = {"ln 3": math.log(3.0), "ln 2": math.log(2.0), "-ln 2": -math.log(2.0)}
+    a = np.array([named.get(x, x) for x in g["a"]], dtype=np.float64)
+    b = np.array(g["b"], dtype=np.float64)
+    nb, B = g["n_blocks"], g["B"]
+    rng = np.random.default_rng(7)
+    qbar = np.stack([math.sqrt(2.0) * a, math.sqrt(2.0) * b], axis=1)
+    kbar = np.stack([np.arange(nb, dtype=np.float64), np.ones(nb)], axis=1)
+    dq, dk = rng.normal(size=(nb, 2)), rng.normal(size=(nb, 2))
+    q = np.stack([qbar + dq, qbar - dq], axis=1).reshape(nb * B, 2)   # block means are qbar
+    k = np.stack([kbar + dk, kbar - dk], axis=1).reshape(nb * B, 2)
+    frac = lambda x: float(eval(x)) if isinstance(x, str) else float(x)  # noqa: E731
+    P = [[frac(x) for x in row] for row in g["P"]]
+    return g, q, k, P
+
+
+def _pooled_case_holds() -> bool:
+    """The golden pooled matrix and every golden gamma cut, against the oracle."""
+    g, q, k, P = _pooled_case()
+    got = O.pooled_scores(q, k, g["B"])
+    for qb, row in enumerate(P):
+        if not np.allclose(got[qb, : qb + 1], row, rtol=0, atol=1e-12):
+            return False
+        if np.any(got[qb, qb + 1:] != 0.0):
+            return False
+    for cut in g["cuts"]:
+        lists, _, _ = O.pe_select(q, k, g["B"], cut["gamma"])
+        if [x.tolist() for x in lists] != cut["lists"]:
+            return False
+    return True
+
+
+def test_pooled_scores_hand_case():
+    """Non-uniform pooled rows with closed forms (the 1/sqrt(d) scale, the operand order
+    Qbar . Kbar and the inclusive causal mask all show), and three gamma cuts derived by hand."""
+    assert _pooled_case_holds()
+
+
+def _mean_pool(x, B):
+    n = x.shape[0]
+    return np.stack([x[i:min(i + B, n)].mean(axis=0) for i in range(0, n, B)])
+
+
+def _softmax_causal(s):
+    nb = s.shape[0]
+    causal = np.tril(np.ones((nb, nb), dtype=bool))
+    s = np.where(causal, s, -np.inf)
+    e = np.where(causal, np.exp(s - s.max(axis=1, keepdims=True)), 0.0)
+    return e / e.sum(axis=1, keepdims=True)
+
+
+@pytest.mark.parametrize("mistake", ["transposed", "unscaled", "sum_pooled_q", "strict_mask"])
+def test_pooled_scores_hand_case_catches_plausible_mistakes(monkeypatch, mistake):
+    """Each plausible slip in pooled_scores, planted on the CPU, fails the hand case above."""
+    def bad(q, k, B):
+        d = q.shape[1]
+        qb, kb = _mean_pool(q, B), _mean_pool(k, B)
+        if mistake == "transposed":
+            s = (kb @ qb.T) / np.sqrt(d)
+        elif mistake == "unscaled":
+            s = qb @ kb.T
+        elif mistake == "sum_pooled_q":
+            s = (B * qb @ kb.T) / np.sqrt(d)
+        else:  # kb < qb only: the diagonal block left out (row 0 then keeps its one entry)
+            s = (qb @ kb.T) / np.sqrt(d)
+            s = s - np.where(np.eye(s.shape[0], dtype=bool), 1e3, 0.0) * (np.arange(s.shape[0]) > 0)[:, None]
+        return _softmax_causal(s)
+
+    monkeypatch.setattr(O, "pooled_scores", bad)
+    assert not _pooled_case_holds()
+    if mistake == "transposed":
+        # the index lists alone already differ: the gamma = 0.55 and 0.7 cuts keep (4, 1)
+        g, q, k, _ = _pooled_case()
+        got = [[x.tolist() for x in O.pe_select(q, k, g["B"], c["gamma"])[0]] for c in g["cuts"]]
+        assert any(gl != c["lists"] for gl, c in zip(got, g["cuts"]))
