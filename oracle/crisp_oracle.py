@@ -262,7 +262,7 @@ def pe_select(q: np.ndarray, k: np.ndarray, B: int, gamma: float):
 # ----------------------------------------------------------------------------------------------
 # Per-head selection  ([BLOG] per-head flow; [CRISP] §3.2, §4)
 # ----------------------------------------------------------------------------------------------
-JSD_TIE_REL = 1e-4  # routing band of the JSD rule: a_bar comes from fp32 pooled means
+JSD_TIE_REL = TIE_REL  # the routing band is the same 1e-5 relative band as every other threshold
 
 
 def select_head(q: np.ndarray, k: np.ndarray, *, block=128, anchors=128, tau_proxy=0.5,
@@ -285,7 +285,7 @@ def select_head(q: np.ndarray, k: np.ndarray, *, block=128, anchors=128, tau_pro
     if route_rule == "jsd":
         j = jsd(pooled_estimate(q[n - B:], k, B), p_v)
         vs = j >= tau_jsd
-        out.update(jsd=j, route_tie=abs(j - tau_jsd) <= JSD_TIE_REL * max(tau_jsd, j))
+        out.update(jsd=j, route_tie=abs(j - tau_jsd) <= JSD_TIE_REL * tau_jsd)
     else:
         vs = route_is_vs(c, tau_proxy)
         out["route_tie"] = abs(c - tau_proxy) <= TIE_REL * tau_proxy

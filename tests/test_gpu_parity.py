@@ -85,7 +85,7 @@ def test_tiny_workload_selection_and_attention():
     params = crisp.Params()
     idx, ws = run_select(q, k, params)
     sels = PT.oracle_select_heads(q, k, params, [0])
-    PT.compare_selection(idx, sels, w.n // 128)
+    PT.compare_selection(idx, sels, w.n // 128, name="tiny_1h_4k")
     assert int(idx.route[0]) == 1
     o, lse = crisp.sparse_prefill(q, k, v, idx, ws=ws)
     crisp.check_status(ws)
@@ -107,7 +107,7 @@ def test_scaled_workloads_full(name, n):
     idx, ws = run_select(q, k, params)
     heads = list(range(w.h_q))
     sels = PT.oracle_select_heads(q, k, params, heads)
-    PT.compare_selection(idx, sels, n // 128)
+    PT.compare_selection(idx, sels, n // 128, name=f"{name} at n={n}")
     o, lse = crisp.sparse_prefill(q, k, v, idx, ws=ws)
     crisp.check_status(ws)
     blocks = sample_blocks(n // 128, heads, 3, seed=n)
@@ -123,7 +123,7 @@ def test_tiny_block_counts(n, tau):
     params = crisp.Params(tau_proxy=tau)
     idx, ws = run_select(q, k, params)
     sels = PT.oracle_select_heads(q, k, params, [0, 1])
-    PT.compare_selection(idx, sels, n // 128)
+    PT.compare_selection(idx, sels, n // 128, name=f"random n={n} tau={tau}")
     o, lse = crisp.sparse_prefill(q, k, v, idx, ws=ws)
     crisp.check_status(ws)
     nb = n // 128
@@ -154,7 +154,7 @@ def test_min_blocks_variant():
     params = crisp.Params(min_blocks=8)
     idx, _ = run_select(q, k, params)
     sels = PT.oracle_select_heads(q, k, params, list(range(w.h_q)))
-    PT.compare_selection(idx, sels, w.n // 128)
+    PT.compare_selection(idx, sels, w.n // 128, name="min_blocks=8 llama8b_32k at n=4096")
 
 
 def test_pe_uniform_closed_form_on_gpu():
@@ -288,7 +288,7 @@ def test_rule_variants_match_oracle(rule, name, n):
     heads = list(range(w.h_q))
     sels = PT.oracle_select_heads(q, k, params, heads)
     nb = w.n // 128
-    PT.compare_selection(idx, sels, nb)
+    PT.compare_selection(idx, sels, nb, name=f"{rule} {name} at n={n}")
     G = w.h_q // w.h_kv
     if params.route_rule:
         for h in heads:
@@ -313,7 +313,7 @@ def test_flexprefill_full_128k():
     nb = w.n // 128
     heads = [0, 1, 2, 3, 12, 13, 30, 31]
     sels = PT.oracle_select_heads(q, k, params, heads)
-    PT.compare_selection(idx, sels, nb)
+    PT.compare_selection(idx, sels, nb, name="flexprefill llama8b_128k")
     for h in range(w.h_q):
         assert int(idx.route[h]) == int(meta["concentrated"][h])
     PT.assert_attention_ok(PT.compare_attention_blocks(q, k, v, o, lse, all_lists(idx, [0, 2]),
@@ -344,7 +344,7 @@ def test_ragged_selection_and_attention(name, n, rules):
     crisp.check_status(ws)
     heads = list(range(w.h_q))
     sels = PT.oracle_select_heads(q, k, params, heads)
-    PT.compare_selection(idx, sels, nb)
+    PT.compare_selection(idx, sels, nb, name=f"ragged {name} n={n} {rules}")
     G = w.h_q // w.h_kv
     ah = sorted({0, w.h_q // 2, w.h_q - 1})
     blocks = [(h, qb) for h in ah for qb in sorted({0, nb // 2, nb - 2, nb - 1}) if qb >= 0]
@@ -399,7 +399,7 @@ def _full(name, sel_heads, attn_per_head, attn_heads=None, seed=0):
     nb = w.n // 128
     sels = PT.oracle_select_heads(q, k, params, sel_heads)
     log = []
-    PT.compare_selection(idx, sels, nb, log)
+    PT.compare_selection(idx, sels, nb, log, name=name)
     G = w.h_q // w.h_kv
     for h in sel_heads:
         assert int(idx.route[h]) == int(meta["concentrated"][h])
@@ -433,5 +433,7 @@ def test_qwen_128k_full():
     _full("qwen7b_128k", list(range(28)), 1, attn_heads=[0, 4, 5, 6, 27])
 
 
-def test_llama_512k_sampled():
-    _full("llama8b_512k", [0, 1, 2, 3, 29, 31], 1, attn_heads=[0, 2, 31])
+def test_llama_512k_all_heads():
+    """Selection of every head at 512k against the oracle (the PE heads' global cuts run over
+    8,390,656 pooled entries each); attention on sampled query blocks of three heads."""
+    _full("llama8b_512k", list(range(32)), 1, attn_heads=[0, 2, 31])
