@@ -184,6 +184,28 @@ def random_qkv(h_q: int, h_kv: int, n: int, d: int = 128, seed: int = 0, device=
     return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
 
 
+def spiked_qkv(h_q: int, h_kv: int, n: int, spike_blocks, gaps, d: int = 128, seed: int = 0, device="cpu",
+               q_rows=None):
+    """N(0,1) bf16 tensors with one planted direction u (|u|^2 = sqrt(d)): every key of the
+    `spike_blocks` gets +w_k u and the queries of head h get +(gaps[h] / w_k) u, so that head's
+    logits against the spiked keys rise by gaps[h] nats (q . k / sqrt(d) grows by w_q w_k).
+    `q_rows` limits the query term to a row range (e.g. the last 128 rows). Edge-case inputs for
+    the softmax reference handling: a spike far above the first key block a walk meets."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    q = torch.randn(h_q, n, d, generator=g)
+    k = torch.randn(h_kv, n, d, generator=g)
+    v = torch.randn(h_kv, n, d, generator=g)
+    u = _planted_direction(g, d, "cpu")
+    w_k = 8.0
+    for kb in spike_blocks:
+        k[:, kb * BLOCK:min(n, (kb + 1) * BLOCK)] += w_k * u
+    lo, hi = q_rows if q_rows is not None else (0, n)
+    for h in range(h_q):
+        q[h, lo:hi] += (float(gaps[h]) / w_k) * u
+    return tuple(t.to(torch.bfloat16).to(device) for t in (q, k, v))
+
+
 def proxy_flops(w: Workload) -> float:
     """Tensor FLOPs of the proxy logits (last query block against all keys) for one layer."""
     return 2.0 * w.h_q * BLOCK * w.n * w.d
@@ -194,5 +216,5 @@ def block_pair_flops(d: int = 128) -> float:
     return 4.0 * BLOCK * BLOCK * d
 
 
-__all__ = ["Workload", "WORKLOADS", "DEFAULT_PARAMS", "generate", "random_qkv",
+__all__ = ["Workload", "WORKLOADS", "DEFAULT_PARAMS", "generate", "random_qkv", "spiked_qkv",
            "concentrated_heads", "proxy_flops", "block_pair_flops", "BLOCK"]
