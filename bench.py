@@ -33,8 +33,9 @@ from dynamic_block_sparse_proxy_b200 import workloads as W  # noqa: E402
 
 METRIC = "prefill tokens/s per layer (select+sparse attn) at 128k; % bf16 peak, % HBM BW"
 DEFAULT_WORKLOAD = "llama8b_128k"
-# kernels per step: proxy pass, 3 for routing, 8 for the PE cut, 5 for the merge, attention
-KERNELS_PER_STEP = 18
+# kernels per step: proxy pass, routing, 5 for the PE path (Q_bar, scores, row softmax, two
+# histogram levels), 3 for the merge, attention
+KERNELS_PER_STEP = 11
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -245,33 +246,37 @@ def run_crisp(args):
     total_s = float(t_step.sum())
     total_s = max_over_ranks(total_s, world, dev)
 
-    # end to end through the public API: pinned host inputs -> device, prefill, output -> host
+    # dense causal attention with the same kernel on the same inputs (after the timed region)
+    dense = None
+    if args.dense:
+        od = torch.empty_like(q)
+        lsed = torch.empty_like(lse)
+        crisp.dense_prefill(q, k, v, o=od, lse=lsed, ws=ws)
+        d_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.dense_steps)]
+        sampler_d = ClockSampler(local)
+        torch.cuda.synchronize()
+        sampler_d.start()
+        time.sleep(0.3)
+        for e0, e1 in d_ev:
+            flush.fill_(7)
+            e0.record(stream)
+            crisp.dense_prefill(q, k, v, o=od, lse=lsed, ws=ws)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        clocks_d = sampler_d.stop()
+        crisp.check_status(ws, "dense")
+        dense_s = float(np.mean([e0.elapsed_time(e1) for e0, e1 in d_ev])) / 1e3
+        dense = {"dense_attn_ms": dense_s * 1e3, "dense_pairs": w.h_q * nb * (nb + 1) // 2,
+                 "dense_tflops": attn_flops(w.h_q * nb * (nb + 1) // 2, w.d) / dense_s / 1e12,
+                 "steps": args.dense_steps, "clocks": clocks_d}
+        del od, lsed
+
     e2e = None
     if args.e2e:
-        qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
-        oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        e_steps = max(1, min(args.steps, 3))
-        for it in range(e_steps + 1):
-            if it == 1:
-                torch.cuda.synchronize()
-                e0 = torch.cuda.Event(enable_timing=True)
-                e1 = torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-            qd.copy_(qh, non_blocking=True)
-            kd.copy_(kh, non_blocking=True)
-            vd.copy_(vh, non_blocking=True)
-            crisp.prefill(qd, kd, vd, params, index=idx, o=o, lse=lse, ws=ws)
-            oh.copy_(o, non_blocking=True)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        crisp.check_status(ws, "e2e")
-        e2e_s = e0.elapsed_time(e1) / 1e3 / e_steps
-        e2e_s = max_over_ranks(e2e_s, world, dev)
-        h2d = (q.numel() + k.numel() + v.numel()) * 2
-        d2h = o.numel() * 2
-        e2e = {"value": job_tokens_per_s(world, w.n, 1, e2e_s), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_s * 1e3}
+        e2e = e2e_pipelined(w, q, k, v, params, idx, ws, max(2, min(args.steps, 4)), dev, stream)
+        e2e_s = max_over_ranks(e2e.pop("seconds_per_step"), world, dev)
+        e2e.update(value=job_tokens_per_s(world, w.n, 1, e2e_s), ms_per_step=e2e_s * 1e3)
 
     if rank != 0:
         if world > 1:
@@ -315,11 +320,84 @@ def run_crisp(args):
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": clocks,
     }
+    if dense is not None:
+        dense["sparse_attn_ms"] = mean_att * 1e3
+        dense["sparse_step_ms"] = (mean_att + mean_sel) * 1e3
+        dense["attn_speedup"] = dense["dense_attn_ms"] / (mean_att * 1e3)
+        dense["step_speedup"] = dense["dense_attn_ms"] / ((mean_att + mean_sel) * 1e3)
+        out["sparse_vs_dense"] = dense
     if args.cpu_baseline:
         out["cpu_baseline"] = oracle_baseline(w, q, k, v, idx, args.cpu_seconds, params=params)
     print(json.dumps(out), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------- end to end
+def e2e_pipelined(w, q, k, v, params, idx, ws, steps: int, dev, stream) -> dict:
+    """The metric end to end through the public API with host buffers: every step copies its Q, K
+    and V from pinned host memory, selects (crisp.select), attends one kv-group at a time
+    (crisp.sparse_prefill on the group's heads and index rows) and copies each group's output back
+    to pinned host memory as soon as that group is done. Two sets of device inputs and outputs let
+    step i+1's uploads run during step i's attention, as a prefill pipeline over layers would; one
+    warm-up step, then `steps` timed steps from the first upload to the last download."""
+    G = w.h_q // w.h_kv
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    oh = [torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(2)]
+    qd = [torch.empty_like(q) for _ in range(2)]
+    kd = [torch.empty_like(k) for _ in range(2)]
+    vd = [torch.empty_like(v) for _ in range(2)]
+    od = [torch.empty_like(q) for _ in range(2)]
+    lsed = [torch.empty(w.h_q, w.n, device=dev, dtype=torch.float32) for _ in range(2)]
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    in_free = [None, None]   # attention of the last step that read input buffer b
+    out_free = [None, None]  # download of the last step that wrote output buffer b
+    gidx = [crisp.Index(idx.route[g * G:(g + 1) * G], idx.c_struct[g * G:(g + 1) * G],
+                        idx.row_ptr[g * G:(g + 1) * G], idx.cols[g * G:(g + 1) * G]) for g in range(w.h_kv)]
+    total = steps + 1
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    for i in range(total):
+        b = i % 2
+        if i == 1:
+            t0.record(up)  # timed region starts with step 1's first upload
+        with torch.cuda.stream(up):
+            if in_free[b] is not None:
+                up.wait_event(in_free[b])
+            qd[b].copy_(qh, non_blocking=True)
+            kd[b].copy_(kh, non_blocking=True)
+            vd[b].copy_(vh, non_blocking=True)
+            ready = torch.cuda.Event()
+            ready.record(up)
+        stream.wait_event(ready)
+        if out_free[b] is not None:
+            stream.wait_event(out_free[b])
+        crisp.select(qd[b], kd[b], params, index=idx, ws=ws)
+        for g in range(w.h_kv):
+            hs = slice(g * G, (g + 1) * G)
+            crisp.sparse_prefill(qd[b][hs], kd[b][g:g + 1], vd[b][g:g + 1], gidx[g], o=od[b][hs], lse=lsed[b][hs],
+                                 ws=ws)
+            done = torch.cuda.Event()
+            done.record(stream)
+            down.wait_event(done)
+            with torch.cuda.stream(down):
+                oh[b][hs].copy_(od[b][hs], non_blocking=True)
+        in_free[b] = torch.cuda.Event()
+        in_free[b].record(stream)
+        out_free[b] = torch.cuda.Event()
+        out_free[b].record(down)
+    down.wait_stream(stream)
+    t1.record(down)
+    torch.cuda.synchronize()
+    crisp.check_status(ws, "e2e")
+    h2d = (q.numel() + k.numel() + v.numel()) * 2
+    d2h = q.numel() * 2
+    return {"unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "seconds_per_step": t0.elapsed_time(t1) / 1e3 / steps, "steps": steps,
+            "how": "pinned host Q/K/V uploaded and O downloaded inside the timed region every step; "
+                   "uploads of step i+1 overlap step i's attention (two device buffer sets), O is "
+                   "downloaded per kv-group as each group's attention finishes"}
 
 
 # ---------------------------------------------------------------------------- CPU oracle arm
@@ -431,6 +509,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--no-dense", dest="dense", action="store_false",
+                    help="skip the dense-attention comparison run after the timed region")
+    ap.add_argument("--dense-steps", type=int, default=2)
     ap.add_argument("--n", type=int, default=0, help="run the workload's generator at another length")
     args = ap.parse_args()
     if args.impl == "reference":

@@ -25,6 +25,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+}  // namespace
+
 // 3D bf16 view [heads][n][128] (heads `ld` rows apart) with 64x128x1 boxes: a head's rows past n
 // read as zeros, so a partial last block never sees the next head's (or sequence's) rows.
 int make_map3(CUtensorMap* m, const void* base, uint64_t n, uint64_t heads, uint64_t ld) {
@@ -40,7 +42,9 @@ int make_map3(CUtensorMap* m, const void* base, uint64_t n, uint64_t heads, uint
   return r == CUDA_SUCCESS ? CRISP_OK : CRISP_ERR_CUDA;
 }
 
+namespace {
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+}  // namespace
 
 // Any n >= 1 (a partial last block when n is not a multiple of 128); selection adds n >= 128.
 int check_shape(int h_q, int h_kv, int n, int d, Shape* s) {
@@ -73,6 +77,7 @@ int check_params(const crisp_params* p) {
   return CRISP_OK;
 }
 
+namespace {
 int check_index(const crisp_index* idx, bool need_select_fields) {
   if (idx == nullptr || idx->row_ptr == nullptr || idx->cols == nullptr) return CRISP_ERR_INVALID_ARG;
   if (need_select_fields && (idx->route == nullptr || idx->c_struct == nullptr)) return CRISP_ERR_INVALID_ARG;
@@ -91,8 +96,10 @@ T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
+}  // namespace
+
 int run_select(const void* q, const void* k, const Shape& s, const crisp_params* p, const crisp_index& out,
-               void* ws, cudaStream_t st) {
+               void* ws, int* status, cudaStream_t st) {
   const Workspace w = workspace_layout(s);
   SelectArgs a{};
   a.s = s;
@@ -104,7 +111,7 @@ int run_select(const void* q, const void* k, const Shape& s, const crisp_params*
   a.tau_jsd = p->tau_jsd;
   a.vs_rule = p->vs_rule;
   a.floor_rule = p->floor_rule;
-  a.status = at<int>(ws, w.status);
+  a.status = status != nullptr ? status : at<int>(ws, w.status);
   a.trace = at<unsigned long long>(ws, w.trace);
   a.part = at<float2>(ws, w.part);
   a.chunk_max = at<float>(ws, w.chunk_max);
@@ -116,11 +123,13 @@ int run_select(const void* q, const void* k, const Shape& s, const crisp_params*
   a.ps_x = at<double>(ws, w.ps_x);
   a.rec_extra = at<float>(ws, w.rec_extra);
   a.kbar = at<float>(ws, w.kbar);
-  a.qbar = at<float>(ws, w.qbar);
+  a.kparts = at<__nv_bfloat16>(ws, w.kparts);
+  a.qparts = at<__nv_bfloat16>(ws, w.qparts);
   a.pbuf = at<float>(ws, w.pbuf);
   a.hist_cnt = at<uint32_t>(ws, w.hist_cnt);
   a.hist_mass = at<unsigned long long>(ws, w.hist_mass);
   a.cut = at<CutState>(ws, w.cut);
+  a.cut_done = at<uint32_t>(ws, w.cut_done);
   a.keep_v = at<uint8_t>(ws, w.keep_v);
   a.keep_s = at<uint8_t>(ws, w.keep_s);
   a.cnt = at<int>(ws, w.cnt);
@@ -134,22 +143,26 @@ int run_select(const void* q, const void* k, const Shape& s, const crisp_params*
   a.cols = out.cols;
   a.debug = out.debug;
 
-  CUtensorMap qm, km;
+  // Q and K as the inputs lay them out; the pooled-block terms as [heads x 3][N_b][128].
+  CUtensorMap qm, km, qpm, kpm;
   int rc = make_map3(&qm, q, (uint64_t)s.n, (uint64_t)s.h_q, (uint64_t)s.ld);
   if (rc == CRISP_OK) rc = make_map3(&km, k, (uint64_t)s.n, (uint64_t)s.h_kv, (uint64_t)s.ld);
+  if (rc == CRISP_OK) rc = make_map3(&qpm, a.qparts, (uint64_t)s.nb, (uint64_t)s.h_q * 3, (uint64_t)s.nb);
+  if (rc == CRISP_OK) rc = make_map3(&kpm, a.kparts, (uint64_t)s.nb, (uint64_t)s.h_kv * 3, (uint64_t)s.nb);
   if (rc != CRISP_OK) return rc;
 
-  // The radix histograms accumulate with atomics: start from zero.
-  if (cudaMemsetAsync(a.hist_cnt, 0, (size_t)s.h_q * kHistBins * 4, st) != cudaSuccess ||
-      cudaMemsetAsync(a.hist_mass, 0, (size_t)s.h_q * kHistBins * 8, st) != cudaSuccess ||
-      cudaMemsetAsync(a.cut, 0, (size_t)s.h_q * sizeof(CutState), st) != cudaSuccess)
+  // The radix histograms accumulate with atomics and the cut levels count finished CTAs: start
+  // from zero (the four arrays are contiguous).
+  if (cudaMemsetAsync(at<uint8_t>(ws, w.hist_cnt), 0, w.cut_done + (size_t)s.h_q * 4 - w.hist_cnt, st) != cudaSuccess)
     return CRISP_ERR_CUDA;
   if (launch_proxy_pass(qm, km, a, st) != cudaSuccess) return CRISP_ERR_CUDA;
   if (launch_route_threshold(a, st) != cudaSuccess) return CRISP_ERR_CUDA;
-  if (launch_pe(a, st) != cudaSuccess) return CRISP_ERR_CUDA;
+  if (launch_pe(a, qpm, kpm, st) != cudaSuccess) return CRISP_ERR_CUDA;
   if (launch_merge(a, st) != cudaSuccess) return CRISP_ERR_CUDA;
   return CRISP_OK;
 }
+
+namespace {
 
 int run_attention(const void* q, const void* k, const void* v, const Shape& s, const int32_t* row_ptr,
                   const int32_t* cols, const int32_t* route, int dense, void* o, float* lse, void* ws,
@@ -219,7 +232,7 @@ int crisp_select(const void* q, const void* k, int h_q, int h_kv, int n, int d, 
   if (rc == CRISP_OK) rc = check_index(out, true);
   if (rc == CRISP_OK) rc = check_ws(ws, ws_bytes, s);
   if (rc != CRISP_OK) return rc;
-  return run_select(q, k, s, params, *out, ws, static_cast<cudaStream_t>(stream));
+  return run_select(q, k, s, params, *out, ws, nullptr, static_cast<cudaStream_t>(stream));
 }
 
 int crisp_sparse_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv, int n, int d,
@@ -259,7 +272,7 @@ int crisp_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv
     idx.debug = nullptr;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  rc = run_select(q, k, s, params, idx, ws, st);
+  rc = run_select(q, k, s, params, idx, ws, nullptr, st);
   if (rc != CRISP_OK) return rc;
   return run_attention(q, k, v, s, idx.row_ptr, idx.cols, idx.route, 0, o, lse, ws, st);
 }
@@ -308,7 +321,7 @@ int crisp_prefill_varlen(const void* q, const void* k, const void* v, int h_q, i
     const auto* ks = static_cast<const __nv_bfloat16*>(k) + off;
     const auto* vs = static_cast<const __nv_bfloat16*>(v) + off;
     auto* os = static_cast<__nv_bfloat16*>(o) + off;
-    rc = run_select(qs, ks, s, params, idx, ws, st);
+    rc = run_select(qs, ks, s, params, idx, ws, nullptr, st);
     if (rc == CRISP_OK) rc = run_attention(qs, ks, vs, s, idx.row_ptr, idx.cols, idx.route, 0, os,
                                            lse != nullptr ? lse + beg : nullptr, ws, st);
     if (rc != CRISP_OK) return rc;

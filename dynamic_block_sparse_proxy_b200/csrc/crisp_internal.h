@@ -15,8 +15,8 @@ namespace crisp {
 constexpr int kB = 128;        // block size (queries and keys)
 constexpr int kD = 128;        // head dimension
 constexpr int kProxyChunk = 16;  // key blocks per proxy CTA
-constexpr int kHistBins = 2048;
-constexpr int kMaxSelectBlocks = 8192;  // selection keeps per-head block arrays in shared memory  // radix-select bins per pass (11, 10, 10 bits)
+constexpr int kHistBins = 2048;        // radix-select bins of the first pass (11, 10, 10 bits)
+constexpr int kMaxSelectBlocks = 8192;  // selection keeps per-head block arrays in shared memory
 constexpr double kMassUnit = 1099511627776.0;  // 2^40: fixed-point scale of histogram masses
 
 struct Shape {
@@ -38,9 +38,9 @@ struct CutState {
 };
 
 struct Workspace {
-  size_t status, trace, part, chunk_max, chunk_tot, row_w, pv, ps_lo, ps_hi, ps_x, rec_extra, kbar, qbar, pbuf,
-      hist_cnt, hist_mass, cut,
-      keep_v, keep_s, cnt, eqcnt, eqbase, selmask, idx_route, idx_c, idx_row_ptr, idx_cols, total;
+  size_t status, trace, part, chunk_max, chunk_tot, row_w, pv, ps_lo, ps_hi, ps_x, rec_extra, kbar, kparts, qparts,
+      pbuf, hist_cnt, hist_mass, cut, cut_done, keep_v, keep_s, cnt, eqcnt, eqbase, selmask, idx_route, idx_c,
+      idx_row_ptr, idx_cols, total;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -69,11 +69,14 @@ inline Workspace workspace_layout(const Shape& s) {
   w.ps_x = take(hq * nb * 8);
   w.rec_extra = take(hq * kB * 4);
   w.kbar = take((size_t)s.h_kv * nb * kD * 4);
-  w.qbar = take(hq * nb * kD * 4);
+  w.kparts = take((size_t)s.h_kv * 3 * nb * kD * 2);
+  w.qparts = take(hq * 3 * nb * kD * 2);
   w.pbuf = take(hq * (size_t)s.cap * 4);
+  // hist_cnt .. cut_done are contiguous: one memset clears them at the start of a selection
   w.hist_cnt = take(hq * kHistBins * 4);
   w.hist_mass = take(hq * kHistBins * 8);
   w.cut = take(hq * sizeof(CutState));
+  w.cut_done = take(hq * 4);
   w.keep_v = take(hq * nb);
   w.keep_s = take(hq * nb);
   w.cnt = take(hq * nb * 4);
@@ -108,12 +111,14 @@ struct SelectArgs {
   double* ps_hi;   // ... and from the keys above it
   double* ps_x;    // ... and (n not a multiple of 128) the next offset block down
   float* rec_extra;  // per proxy row: recency-window mass inside block N_b-2 (n not a multiple of 128)
-  float* kbar;
-  float* qbar;
+  float* kbar;                  // K_bar fp32 [h_kv][N_b][128]
+  __nv_bfloat16* kparts;        // K_bar as three bf16 terms [h_kv][3][N_b][128] (sum exact)
+  __nv_bfloat16* qparts;        // Q_bar of PE heads, likewise [h_q][3][N_b][128]
   float* pbuf;
   uint32_t* hist_cnt;
   unsigned long long* hist_mass;  // fixed point, 2^-40 units
   CutState* cut;
+  uint32_t* cut_done;           // per head: CTAs of the current radix level that finished
   uint8_t* keep_v;
   uint8_t* keep_s;
   int* cnt;
@@ -145,10 +150,19 @@ struct AttnArgs {
 cudaError_t launch_proxy_pass(const CUtensorMap& q_map, const CUtensorMap& k_map, const SelectArgs& a,
                               cudaStream_t st);
 cudaError_t launch_route_threshold(const SelectArgs& a, cudaStream_t st);
-cudaError_t launch_pe(const SelectArgs& a, cudaStream_t st);
+cudaError_t launch_pe(const SelectArgs& a, const CUtensorMap& qp_map, const CUtensorMap& kp_map, cudaStream_t st);
 cudaError_t launch_merge(const SelectArgs& a, cudaStream_t st);
 cudaError_t launch_sparse_attn(const CUtensorMap& q_map, const CUtensorMap& k_map,
                                const CUtensorMap& v_map, const AttnArgs& a, cudaStream_t st);
 cudaError_t launch_timeout_selftest(int* status, unsigned long long limit_ns, cudaStream_t st);
+
+// Host-side helpers shared by the entry points (crisp_api.cu).
+int check_shape(int h_q, int h_kv, int n, int d, Shape* s);
+int check_params(const crisp_params* p);
+int make_map3(CUtensorMap* m, const void* base, uint64_t n, uint64_t heads, uint64_t ld);
+// The selection launch sequence on the workspace at `ws` (at least workspace_layout(s).total
+// bytes, 256-byte aligned). `status`, when not null, replaces the workspace's status word.
+int run_select(const void* q, const void* k, const Shape& s, const crisp_params* p, const crisp_index& out,
+               void* ws, int* status, cudaStream_t st);
 
 }  // namespace crisp

@@ -2,19 +2,24 @@
 // attention A_hat = softmax(Q_hat K^T / sqrt(d)) over a representative query subset, here the
 // last query block; §4: vertical = column means, slash = diagonal means, pooled into blocks).
 //
-// One CTA handles two q-heads of one GQA group (two "tiles": their last query blocks) against a
-// chunk of kProxyChunk key blocks of the shared kv-head, so every K block is read once for both.
-//   warp 8      TMA producer: both Q tiles, then the chunk's K blocks through a 3-stage ring;
+// Work item: two q-heads of one GQA group (two "tiles": their last query blocks) against a chunk
+// of kProxyChunk key blocks of the shared kv-head, so every K block is read once for both. The
+// grid is persistent (one CTA per SM): CTA c takes a contiguous run of the items listed pair by
+// pair, so a CTA's items mostly share their Q tiles, and the barrier rings run on from one item
+// to the next.
+//   warp 8      TMA producer: the two Q tiles whenever the pair changes (after the MMAs that read
+//               the old ones), then the chunks' K blocks through a 3-stage ring;
 //   warp 9      one thread issues S_t = Q_t K_blk^T (128x128x128, bf16 -> fp32) into a
 //               double-buffered TMEM tile per head;
-//   warps 0-7   softmax, one warpgroup per head, one proxy row per thread: read the S row with
-//               one TMEM round trip, mask the keys the causal limit cuts (key j visible to row r
-//               iff j <= n-B+r), and accumulate exp2(x - m) against a lagging row reference m (set
-//               by the chunk's first block, moved only when a block's sum would leave
-//               [0, 2^64]) into two sums per key block: keys at or below the row's diagonal
-//               offset (t <= r) and above it (t > r);
+//   warps 0-7   softmax, one warpgroup per head, one proxy row per thread: read the S row from
+//               TMEM 32 columns at a time (the next load in flight while the current columns are
+//               exponentiated), mask the keys the causal limit cuts (key j visible to row r iff
+//               j <= n-B+r), and accumulate exp2(x - m) against a lagging row reference m (set
+//               by the chunk's first block, moved only when a block's sum would leave [0, 2^64])
+//               into two sums per key block: keys at or below the row's diagonal offset (t <= r)
+//               and above it (t > r);
 //   warps 10-11 sum rows of each K block into the mean-pooled key K_bar of the PE path; the
-//               CTAs of one group share the 16 column chunks between them.
+//               items of one group share the 16 column chunks between them.
 // A key at offset t of block kb seen by proxy row r lies on diagonal offset (N_b-1-kb)*B + (r-t),
 // so the first sum belongs to slash block N_b-1-kb and the second to N_b-2-kb; their total is
 // the block's vertical mass. When n is not a multiple of 128 (t_last keys in the last block) the
@@ -41,6 +46,7 @@ struct __align__(1024) ProxySmem {
   __nv_bfloat16 k[NS][kB * kD];
   float2 part[2][kProxyChunk][kB];  // per tile, block and row: (lower, upper) sums
   uint64_t q_full;
+  uint64_t q_empty;
   uint64_t k_full[NS];
   uint64_t k_empty[NS];
   uint64_t s_full[2][2];
@@ -55,6 +61,103 @@ __device__ __forceinline__ void fail(ProxySmem& sm, int* status) {
   *reinterpret_cast<volatile int*>(&sm.abort) = 1;
 }
 
+// tcgen05.wait::ld that also names the destination registers of the load it waits for, so the
+// compiler cannot move their first use above the wait.
+__device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+        "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+        "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+        "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+        "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
+}
+
+// Item `it` of the pair-major list: (pair, chunk) and what follows from them.
+struct Item {
+  int pair, chunk, kv, pig, h0, ntiles, kb0, nblk;
+  __device__ __forceinline__ Item(const Shape& s, int it) {
+    const int ppg = (s.G + 1) / 2;
+    pair = it / s.n_chunks;
+    chunk = it % s.n_chunks;
+    kv = pair / ppg;
+    pig = pair % ppg;
+    h0 = kv * s.G + 2 * pig;
+    ntiles = (2 * pig + 1 < s.G) ? 2 : 1;
+    kb0 = chunk * kProxyChunk;
+    nblk = min(kProxyChunk, s.nb - kb0);
+  }
+};
+
+// One block of one row, the common case (n a multiple of 128, not the last block): S read 32
+// columns at a time (the next load in flight while these are exponentiated), and the row's sums
+// below/above its diagonal column r (warp `grp` holds rows 32grp..32grp+31, so columns
+// of chunk c < grp are all below, c > grp all above, and chunk grp splits at the lane).
+__device__ __forceinline__ void block_sums_fast(uint32_t sbase, float nm, int grp, int lane, float& lo, float& hi) {
+  uint32_t v[2][32];
+  lo = 0.f;
+  hi = 0.f;
+  tmem_ld32(sbase, v[0]);
+  tmem_ld_wait_regs(v[0]);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t(&x)[32] = v[c & 1];
+    if (c < 3) tmem_ld32(sbase + (c + 1) * 32, v[(c + 1) & 1]);
+    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int q = 0; q < 32; ++q) {
+      const float e = fast_exp2(fmaf(__uint_as_float(x[q]), kScaleLog2, nm));
+      x[q] = __float_as_uint(e);
+      s4[q & 3] += e;
+    }
+    const float sc = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+    if (c < grp) {
+      lo += sc;
+    } else if (c > grp) {
+      hi += sc;
+    } else {
+      float l2[2] = {0.f, 0.f}, h2[2] = {0.f, 0.f};
+#pragma unroll
+      for (int q = 0; q < 32; ++q) {
+        const float e = __uint_as_float(x[q]);
+        if (q <= lane) l2[q & 1] += e; else h2[q & 1] += e;
+      }
+      lo += l2[0] + l2[1];
+      hi += h2[0] + h2[1];
+    }
+    if (c < 3) tmem_ld_wait_regs(v[(c + 1) & 1]);
+  }
+}
+
+// Largest logit of the row in this block (after the causal mask), scaled to log2 units.
+__device__ __forceinline__ float block_max_scaled(uint32_t sbase, int lim, bool edge) {
+  uint32_t v[2][32];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    tmem_ld32(sbase + h * 64, v[0]);
+    tmem_ld32(sbase + h * 64 + 32, v[1]);
+    tmem_ld_wait_regs(v[0]);
+    tmem_ld_wait_regs(v[1]);
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int q = 0; q < 32; q += 2) {
+        float a = __uint_as_float(v[c][q]), b = __uint_as_float(v[c][q + 1]);
+        if (edge) {
+          if (h * 64 + c * 32 + q > lim) a = -INFINITY;
+          if (h * 64 + c * 32 + q + 1 > lim) b = -INFINITY;
+        }
+        float m3;
+        asm("max.f32 %0, %1, %2, %3;" : "=f"(m3) : "f"(mx), "f"(a), "f"(b));
+        mx = m3;
+      }
+  }
+  return mx * kScaleLog2;
+}
+
 // RAGGED: n is not a multiple of 128 (separate instance, so the common case keeps the lane-aligned
 // split with no extra work in its exponential loop).
 template <bool RAGGED>
@@ -67,21 +170,16 @@ __global__ void __launch_bounds__(THREADS, 1)
   const volatile int* abort = &sm.abort;
 
   const Shape& s = a.s;
-  const int pairs_per_group = (s.G + 1) / 2;
-  const int n_pairs = s.h_kv * pairs_per_group;
-  const int pair = blockIdx.x % n_pairs;
-  const int chunk = blockIdx.x / n_pairs;
-  const int kv = pair / pairs_per_group;
-  const int pig = pair % pairs_per_group;  // pair index within its group
-  const int h0 = kv * s.G + 2 * pig;
-  const int ntiles = (2 * pig + 1 < s.G) ? 2 : 1;
-  const int kb0 = chunk * kProxyChunk;
-  const int nblk = min(kProxyChunk, s.nb - kb0);
+  const int ppg = (s.G + 1) / 2;
+  const int n_items = s.h_kv * ppg * s.n_chunks;
+  const int it0 = (int)((long long)blockIdx.x * n_items / gridDim.x);
+  const int it1 = (int)((long long)(blockIdx.x + 1) * n_items / gridDim.x);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.q_full, 1);
+    mbar_init(&sm.q_empty, 1);
     for (int i = 0; i < NS; ++i) {
       mbar_init(&sm.k_full[i], 1);
       mbar_init(&sm.k_empty[i], 3);  // MMA commit + two pooling warps
@@ -110,66 +208,97 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       tma_prefetch_desc(&q_map);
       tma_prefetch_desc(&k_map);
-      mbar_arrive_expect_tx(&sm.q_full, TILE_BYTES * ntiles);
-      for (int t = 0; t < ntiles; ++t) {  // the last 128 queries of each head
-        tma_load_3d(&q_map, &sm.q_full, sm.q[t], 0, s.n - kB, h0 + t);
-        tma_load_3d(&q_map, &sm.q_full, sm.q[t] + kB * 64, 64, s.n - kB, h0 + t);
-      }
-      int issued = 0;
-      for (int j = 0; j < nblk; ++j) {
-        const int st = j % NS;
-        if (!mbar_wait(&sm.k_empty[st], ((j / NS) & 1) ^ 1, abort)) {
-          fail(sm, a.status);
-          break;
+      int kc = 0, qn = 0, prev_pair = -1;
+      bool ok = true;
+      for (int it = it0; ok && it < it1; ++it) {
+        const Item w(s, it);
+        if (w.pair != prev_pair) {
+          // the last 128 queries of each head, once the MMAs on the previous pair's tiles are done
+          if (qn > 0 && !mbar_wait(&sm.q_empty, (qn - 1) & 1, abort)) {
+            fail(sm, a.status);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&sm.q_full, TILE_BYTES * w.ntiles);
+          for (int t = 0; t < w.ntiles; ++t) {
+            tma_load_3d(&q_map, &sm.q_full, sm.q[t], 0, s.n - kB, w.h0 + t);
+            tma_load_3d(&q_map, &sm.q_full, sm.q[t] + kB * 64, 64, s.n - kB, w.h0 + t);
+          }
+          ++qn;
+          prev_pair = w.pair;
         }
-        const int ky = (kb0 + j) * kB;  // rows past n of a partial last block arrive as zeros
-        mbar_arrive_expect_tx(&sm.k_full[st], TILE_BYTES);
-        tma_load_3d(&k_map, &sm.k_full[st], sm.k[st], 0, ky, kv);
-        tma_load_3d(&k_map, &sm.k_full[st], sm.k[st] + kB * 64, 64, ky, kv);
-        ++issued;
+        for (int j = 0; j < w.nblk; ++j, ++kc) {
+          const int st = kc % NS;
+          if (!mbar_wait(&sm.k_empty[st], ((kc / NS) & 1) ^ 1, abort)) {
+            fail(sm, a.status);
+            ok = false;
+            break;
+          }
+          const int ky = (w.kb0 + j) * kB;  // rows past n of a partial last block arrive as zeros
+          mbar_arrive_expect_tx(&sm.k_full[st], TILE_BYTES);
+          tma_load_3d(&k_map, &sm.k_full[st], sm.k[st], 0, ky, w.kv);
+          tma_load_3d(&k_map, &sm.k_full[st], sm.k[st] + kB * 64, 64, ky, w.kv);
+        }
       }
       // Never leave with copies in flight: wait (bounded) for the last load of each stage.
-      mbar_wait(&sm.q_full, 0, nullptr);
-      for (int j = max(0, issued - NS); j < issued; ++j) mbar_wait(&sm.k_full[j % NS], (j / NS) & 1, nullptr);
+      if (qn > 0) mbar_wait(&sm.q_full, (qn - 1) & 1, nullptr);
+      for (int j = max(0, kc - NS); j < kc; ++j) mbar_wait(&sm.k_full[j % NS], (j / NS) & 1, nullptr);
     }
     __syncwarp();
   } else if (warp == MMA_WARP) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
-      bool ok = mbar_wait(&sm.q_full, 0, abort);
-      if (!ok) fail(sm, a.status);
-      for (int j = 0; ok && j < nblk; ++j) {
-        const int st = j % NS, b = j & 1;
-        if (!mbar_wait(&sm.k_full[st], (j / NS) & 1, abort)) {
-          fail(sm, a.status);
-          break;
-        }
-        for (int t = 0; t < ntiles && ok; ++t) {
-          if (!mbar_wait(&sm.s_free[t][b], ((j >> 1) & 1) ^ 1, abort)) {
+      int kc = 0, qn = 0, prev_pair = -1;
+      int tb[2] = {0, 0};  // blocks issued per tile so far (S buffer and phase)
+      bool ok = true;
+      for (int it = it0; ok && it < it1; ++it) {
+        const Item w(s, it);
+        if (w.pair != prev_pair) {
+          if (qn > 0) umma_commit(&sm.q_empty);  // the old Q tiles are free once these MMAs finish
+          if (!mbar_wait(&sm.q_full, qn & 1, abort)) {
             fail(sm, a.status);
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t qa = smem_u32(sm.q[t]), ka = smem_u32(sm.k[st]);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-            umma_ss(tmem + t * 256 + b * 128, desc_kmajor_sw128(qa + off), desc_kmajor_sw128(ka + off), idesc,
-                    kk > 0);
-          }
-          umma_commit(&sm.s_full[t][b]);
+          ++qn;
+          prev_pair = w.pair;
         }
-        if (!ok) break;
-        umma_commit(&sm.k_empty[st]);
+        for (int j = 0; ok && j < w.nblk; ++j, ++kc) {
+          const int st = kc % NS;
+          if (!mbar_wait(&sm.k_full[st], (kc / NS) & 1, abort)) {
+            fail(sm, a.status);
+            ok = false;
+            break;
+          }
+          for (int t = 0; t < w.ntiles; ++t) {
+            const int b = tb[t] & 1;
+            if (!mbar_wait(&sm.s_free[t][b], ((tb[t] >> 1) & 1) ^ 1, abort)) {
+              fail(sm, a.status);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t qa = smem_u32(sm.q[t]), ka = smem_u32(sm.k[st]);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+              umma_ss(tmem + t * 256 + b * 128, desc_kmajor_sw128(qa + off), desc_kmajor_sw128(ka + off), idesc,
+                      kk > 0);
+            }
+            umma_commit(&sm.s_full[t][b]);
+            ++tb[t];
+          }
+          if (!ok) break;
+          umma_commit(&sm.k_empty[st]);
+        }
       }
       // Never release TMEM under a running MMA: wait (bounded) for all issued work.
       umma_commit(&sm.mma_done);
       mbar_wait(&sm.mma_done, 0, nullptr);
     }
     __syncwarp();
-  } else if (warp < 4 * ntiles) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax rows
     const int t = warp >> 2;
     const int grp = warp & 3;
@@ -182,189 +311,184 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int t_last = s.n - (s.nb - 1) * kB;
     constexpr bool ragged = RAGGED;
     const int sigma = (t_last + r) & (kB - 1);
-    float m = -INFINITY;
-    float rec = 0.f;  // recency-window mass in block N_b-2 (columns >= t_last), ragged n only
+    int tb = 0;  // blocks of this tile so far (S buffer and phase)
     bool ok = true;
-    for (int j = 0; j < nblk; ++j) {
-      const int b = j & 1;
-      if (!warp_wait(&sm.s_full[t][b], (j >> 1) & 1, abort)) {
-        fail(sm, a.status);
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      // Exponentials use the row reference m of the chunk's earlier blocks without this block's
-      // maximum (fp32 keeps them exact until they overflow); the first block sets m from its
-      // maximum, and a block whose sum would leave [0, 2^64] is redone against its maximum with
-      // the earlier partial sums rescaled. S stays in TMEM until the block is done.
-      uint32_t v[4][32];
-      const uint32_t sbase = tmem + t * 256 + b * 128 + lane_off;
-      const int kb = kb0 + j;
-      const int lim = s.n - kB + r - kb * kB;  // row r sees columns c <= lim of this block
-      const bool edge = RAGGED ? kb >= s.nb - 2 : kb == s.nb - 1;  // blocks lim can cut
-      const bool rec_blk = ragged && s.nb >= 3 && kb == s.nb - 2;
-      bool need_max = (m == -INFINITY);
-      float lo = 0.f, hi = 0.f, rx = 0.f;
-      for (int attempt = 0; attempt < 2; ++attempt) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(sbase + c * 32, v[c]);
-        tmem_ld_wait();
-        if (edge) {
-          // causal: row r (position n-128+r) sees keys up to its own position only
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int q = 0; q < 32; ++q)
-              if (c * 32 + q > lim) v[c][q] = __float_as_uint(-INFINITY);
+    for (int it = it0; ok && it < it1; ++it) {
+      const Item w(s, it);
+      if (t >= w.ntiles) continue;  // a group's odd last head: this tile has no head here
+      float m = -INFINITY;
+      float rec = 0.f;  // recency-window mass in block N_b-2 (columns >= t_last), ragged n only
+      for (int j = 0; j < w.nblk; ++j, ++tb) {
+        const int b = tb & 1;
+        if (!warp_wait(&sm.s_full[t][b], (tb >> 1) & 1, abort)) {
+          fail(sm, a.status);
+          ok = false;
+          break;
         }
-        if (need_max) {
-          float mx8[8];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) mx8[q] = -INFINITY;
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int q = 0; q < 32; ++q) mx8[q & 7] = fmaxf(mx8[q & 7], __uint_as_float(v[c][q]));
-          const float xm = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * kScaleLog2;
-          if (xm > m) {
-            const float f = fast_exp2(m - xm);  // 0 while m = -inf
-            for (int jj = 0; jj < j; ++jj) {
-              float2 pv = sm.part[t][jj][r];
-              pv.x *= f;
-              pv.y *= f;
-              sm.part[t][jj][r] = pv;
+        tc_fence_after();
+        // Exponentials use the row reference m of the chunk's earlier blocks without this block's
+        // maximum (fp32 keeps them exact until they overflow); the first block sets m from its
+        // maximum, and a block whose sum would leave [0, 2^64] is redone against its maximum with
+        // the earlier partial sums rescaled. S stays in TMEM until the block is done.
+        const uint32_t sbase = tmem + t * 256 + b * 128 + lane_off;
+        const int kb = w.kb0 + j;
+        const int lim = s.n - kB + r - kb * kB;  // row r sees columns c <= lim of this block
+        const bool edge = RAGGED ? kb >= s.nb - 2 : kb == s.nb - 1;  // blocks lim can cut
+        const bool rec_blk = ragged && s.nb >= 3 && kb == s.nb - 2;
+        bool need_max = (m == -INFINITY);
+        float lo = 0.f, hi = 0.f, rx = 0.f;
+        for (int attempt = 0; attempt < 2; ++attempt) {
+          if (need_max) {
+            const float xm = block_max_scaled(sbase, lim, edge);
+            if (xm > m) {
+              const float f = fast_exp2(m - xm);  // 0 while m = -inf
+              for (int jj = 0; jj < j; ++jj) {
+                float2 pv = sm.part[t][jj][r];
+                pv.x *= f;
+                pv.y *= f;
+                sm.part[t][jj][r] = pv;
+              }
+              rec *= f;
+              m = xm;
             }
-            rec *= f;
-            m = xm;
           }
-        }
-        const float nm = -m;
-        // chunks below the warp's group hold keys t <= r, chunks above hold t > r; chunk grp
-        // straddles the diagonal offset lane by lane
-        lo = 0.f;
-        hi = 0.f;
-        rx = 0.f;
-        if constexpr (RAGGED) {
-          // the split column (t_last + r) mod 128 is not aligned with the warp's lanes
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int q = 0; q < 32; ++q) {
-              const int col = c * 32 + q;
-              const float e = fast_exp2(fmaf(__uint_as_float(v[c][q]), kScaleLog2, nm));
-              if (col <= sigma) lo += e; else hi += e;
-              if (rec_blk && col >= t_last) rx += e;
-            }
-        } else {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float s4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            const float e = fast_exp2(fmaf(__uint_as_float(v[c][q]), kScaleLog2, nm));
-            v[c][q] = __float_as_uint(e);
-            s4[q & 3] += e;
-          }
-          const float sc = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-          if (c < grp) {
-            lo += sc;
-          } else if (c > grp) {
-            hi += sc;
+          const float nm = -m;
+          if (!RAGGED && !edge) {
+            block_sums_fast(sbase, nm, grp, lane, lo, hi);
           } else {
-            float l2[2] = {0.f, 0.f}, h2[2] = {0.f, 0.f};
+            // hardware exp2 only, every column tested against the causal limit and (n not a
+            // multiple of 128) the split column, which is not aligned with the lanes
+            lo = 0.f;
+            hi = 0.f;
+            rx = 0.f;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              uint32_t v[32];
+              tmem_ld32(sbase + c * 32, v);
+              tmem_ld_wait_regs(v);
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
-              const float e = __uint_as_float(v[c][q]);
-              if (q <= lane) l2[q & 1] += e; else h2[q & 1] += e;
+              for (int q = 0; q < 32; ++q) {
+                const int col = c * 32 + q;
+                float e = fast_exp2(fmaf(__uint_as_float(v[q]), kScaleLog2, nm));
+                if (edge && col > lim) e = 0.f;  // causal: row r sees keys up to its own position
+                const bool low = RAGGED ? col <= sigma : col <= r;
+                if (low) lo += e; else hi += e;
+                if (rec_blk && col >= t_last) rx += e;
+              }
             }
-            lo += l2[0] + l2[1];
-            hi += h2[0] + h2[1];
           }
+          const bool redo = !need_max && !(lo + hi <= 18446744073709551616.0f);  // 2^64, or inf / nan
+          if (!__any_sync(0xffffffffu, redo)) break;
+          need_max = true;
         }
-        }
-        const bool redo = !need_max && !(lo + hi <= 18446744073709551616.0f);  // 2^64, or inf / nan
-        if (!__any_sync(0xffffffffu, redo)) break;
-        need_max = true;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.s_free[t][b]);
+        sm.part[t][j][r] = make_float2(lo, hi);
+        if (rec_blk) rec = rx;
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.s_free[t][b]);
-      sm.part[t][j][r] = make_float2(lo, hi);
-      if (rec_blk) rec = rx;
-    }
-    if (ok) {
-      const int h = h0 + t;
+      if (!ok) break;
+      const int h = w.h0 + t;
       float tot = 0.f;
-      for (int jj = 0; jj < nblk; ++jj) {
+      for (int jj = 0; jj < w.nblk; ++jj) {
         const float2 pv = sm.part[t][jj][r];
-        a.part[((size_t)h * s.nb + kb0 + jj) * kB + r] = pv;
+        a.part[((size_t)h * s.nb + w.kb0 + jj) * kB + r] = pv;
         tot += pv.x + pv.y;
       }
-      const size_t ci = ((size_t)h * s.n_chunks + chunk) * kB + r;
+      const size_t ci = ((size_t)h * s.n_chunks + w.chunk) * kB + r;
       a.chunk_max[ci] = m;
       a.chunk_tot[ci] = tot;
-      if (ragged && s.nb >= 3 && s.nb - 2 >= kb0 && s.nb - 2 < kb0 + nblk) a.rec_extra[(size_t)h * kB + r] = rec;
+      if (ragged && s.nb >= 3 && s.nb - 2 >= w.kb0 && s.nb - 2 < w.kb0 + w.nblk)
+        a.rec_extra[(size_t)h * kB + r] = rec;
     }
     __syncwarp();
   } else if (warp >= POOL_WARP) {
     // ------------------------------------------------------------------ K block mean (PE path)
-    // Column chunk cc (8 bf16 of each row) belongs to the group's CTA cc % pairs_per_group, and
-    // within the CTA to pooling warp (its slot index) % 2. Lane (slot, row group) sums every
-    // groups-th row of its chunk; shuffles combine the row groups.
+    // Column chunk cc (8 bf16 of each row) belongs to the group's item cc % ppg (by the item's
+    // pair index within its group), and within the item to pooling warp (its slot index) % 2.
+    // Lane (slot, row group) sums every groups-th row of its chunk; shuffles combine the row
+    // groups.
     const int pw = warp - POOL_WARP;
-    const int ncc_cta = (16 - pig + pairs_per_group - 1) / pairs_per_group;
-    const int ncc = (ncc_cta - pw + 1) / 2;
-    int groups = 1;
-    while (groups < 32 && groups * 2 * ncc <= 32) groups *= 2;
-    const int slot = lane / groups;
-    const int rg = lane % groups;
-    const bool active = slot < ncc;
-    const int cc = pig + (2 * slot + pw) * pairs_per_group;
-    const int half = cc >> 3, ch = cc & 7;
-    for (int j = 0; j < nblk; ++j) {
-      const int st = j % NS;
-      if (!warp_wait(&sm.k_full[st], (j / NS) & 1, abort)) {
-        fail(sm, a.status);
-        break;
-      }
-      float acc[8];
+    int kc = 0;
+    bool ok = true;
+    for (int it = it0; ok && it < it1; ++it) {
+      const Item w(s, it);
+      const int ncc_item = (16 - w.pig + ppg - 1) / ppg;
+      const int ncc = (ncc_item - pw + 1) / 2;
+      int groups = 1;
+      while (groups < 32 && groups * 2 * ncc <= 32) groups *= 2;
+      const int slot = lane / groups;
+      const int rg = lane % groups;
+      const bool active = slot < ncc;
+      const int cc = w.pig + (2 * slot + pw) * ppg;
+      const int half = cc >> 3, ch = cc & 7;
+      for (int j = 0; j < w.nblk; ++j, ++kc) {
+        const int st = kc % NS;
+        if (!warp_wait(&sm.k_full[st], (kc / NS) & 1, abort)) {
+          fail(sm, a.status);
+          ok = false;
+          break;
+        }
+        float acc[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-      if (active) {
-        // 128/groups rows per lane, eight independent 16-byte loads in flight
-        const uint8_t* base = reinterpret_cast<const uint8_t*>(sm.k[st]) + half * HALF_BYTES;
-        for (int row0 = rg; row0 < kB; row0 += 8 * groups) {
-          uint4 u[8];
+        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+        if (active) {
+          // 128/groups rows per lane, eight independent 16-byte loads in flight
+          const uint8_t* base = reinterpret_cast<const uint8_t*>(sm.k[st]) + half * HALF_BYTES;
+          for (int row0 = rg; row0 < kB; row0 += 8 * groups) {
+            uint4 u[8];
 #pragma unroll
-          for (int x = 0; x < 8; ++x) {
-            const int row = row0 + x * groups;
-            u[x] = row < kB ? *reinterpret_cast<const uint4*>(base + sw128_offset(row, ch)) : make_uint4(0, 0, 0, 0);
-          }
+            for (int x = 0; x < 8; ++x) {
+              const int row = row0 + x * groups;
+              u[x] = row < kB ? *reinterpret_cast<const uint4*>(base + sw128_offset(row, ch)) : make_uint4(0, 0, 0, 0);
+            }
 #pragma unroll
-          for (int x = 0; x < 8; ++x) {
-            const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&u[x]);
+            for (int x = 0; x < 8; ++x) {
+              const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&u[x]);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float2 f = __bfloat1622float2(p2[i]);
-              acc[2 * i] += f.x;
-              acc[2 * i + 1] += f.y;
+              for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(p2[i]);
+                acc[2 * i] += f.x;
+                acc[2 * i + 1] += f.y;
+              }
             }
           }
         }
-      }
-      for (int o = 1; o < groups; o <<= 1)
+        for (int o = 1; o < groups; o <<= 1)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
-      if (active && rg == 0) {
-        float4* dst = reinterpret_cast<float4*>(a.kbar + ((size_t)kv * s.nb + kb0 + j) * kD + cc * 8);
-        // a partial last block averages the rows it has (the rest arrived as zeros)
-        const float inv = kb0 + j == s.nb - 1 ? 1.f / (float)(s.n - (s.nb - 1) * kB) : 1.f / kB;
-        dst[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-        dst[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+          for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+        if (active && rg == 0) {
+          const size_t kb = (size_t)w.kb0 + j;
+          float4* dst = reinterpret_cast<float4*>(a.kbar + ((size_t)w.kv * s.nb + kb) * kD + cc * 8);
+          // a partial last block averages the rows it has (the rest arrived as zeros)
+          const float inv = kb == (size_t)s.nb - 1 ? 1.f / (float)(s.n - (s.nb - 1) * kB) : 1.f / kB;
+          float mv[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mv[i] = acc[i] * inv;
+          dst[0] = make_float4(mv[0], mv[1], mv[2], mv[3]);
+          dst[1] = make_float4(mv[4], mv[5], mv[6], mv[7]);
+          // the same means as three bf16 terms whose sum is exact (hi, mid, lo), for the
+          // tensor-core pooled scores: [kv][term][N_b][128]
+          uint32_t pk[3][4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            float r0 = mv[2 * i], r1 = mv[2 * i + 1];
+#pragma unroll
+            for (int tt = 0; tt < 3; ++tt) {
+              const __nv_bfloat16 b0 = __float2bfloat16_rn(r0), b1 = __float2bfloat16_rn(r1);
+              pk[tt][i] = (uint32_t)__bfloat16_as_ushort(b0) | ((uint32_t)__bfloat16_as_ushort(b1) << 16);
+              r0 -= __bfloat162float(b0);
+              r1 -= __bfloat162float(b1);
+            }
+          }
+#pragma unroll
+          for (int tt = 0; tt < 3; ++tt)
+            *reinterpret_cast<uint4*>(a.kparts + (((size_t)w.kv * 3 + tt) * s.nb + kb) * kD + cc * 8) =
+                make_uint4(pk[tt][0], pk[tt][1], pk[tt][2], pk[tt][3]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.k_empty[st]);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.k_empty[st]);
     }
     __syncwarp();
   }
@@ -378,6 +502,16 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
+int num_sms() {
+  static int n = [] {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return 148;
+    return v;
+  }();
+  return n;
+}
+
 }  // namespace
 
 cudaError_t launch_proxy_pass(const CUtensorMap& q_map, const CUtensorMap& k_map, const SelectArgs& a,
@@ -387,8 +521,8 @@ cudaError_t launch_proxy_pass(const CUtensorMap& q_map, const CUtensorMap& k_map
   auto kernel = ragged ? proxy_pass_kernel<true> : proxy_pass_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int n_pairs = a.s.h_kv * ((a.s.G + 1) / 2);
-  dim3 grid(n_pairs * a.s.n_chunks);
+  const int n_items = a.s.h_kv * ((a.s.G + 1) / 2) * a.s.n_chunks;
+  dim3 grid(min(n_items, num_sms()));  // persistent: one CTA per SM, a run of items each
   kernel<<<grid, THREADS, smem, st>>>(q_map, k_map, a);
   return cudaGetLastError();
 }

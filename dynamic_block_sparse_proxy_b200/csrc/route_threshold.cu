@@ -1,8 +1,8 @@
 // route_threshold.cu — per-head routing and the Vertical-Slash noise-floor rule.
 //
 // Inputs are the proxy pass's per-(row, key block) split sums, each relative to its chunk's
-// reference row maximum. Three kernels (row statistics, block masses over many CTAs, and one
-// CTA per q-head for the decisions):
+// reference row maximum. One kernel: row statistics and block masses over many CTAs per head,
+// and the head's last CTA takes the decisions:
 //   1. per proxy row r: global max M_r and normaliser Z_r over all chunks, and the weight
 //      w = exp2(m_chunk - M_r) / (Z_r * B) that turns a chunk's sums into column-mean mass;
 //   2. p_v[kb] = sum_r w*(lo+hi) (vertical block mass), and the slash block masses
@@ -66,74 +66,6 @@ __device__ int block_argmax(double v, int idx, double* redv, int* redi) {
     }
   }
   return bi;
-}
-
-// 1. Per proxy row r of head h: global reference max M_r over the chunks, normaliser Z_r, and
-//    the weight w = exp2(m_chunk - M_r) / (Z_r * B) that turns a chunk's sums into column-mean mass.
-//    One warp per row, its lanes across the chunks.
-constexpr int STAT_ROWS = 8;
-__global__ void __launch_bounds__(STAT_ROWS * 32) row_stats_kernel(const SelectArgs a) {
-  const Shape& s = a.s;
-  const int h = blockIdx.y, r = blockIdx.x * STAT_ROWS + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  const float* mc = a.chunk_max + (size_t)h * s.n_chunks * kB;
-  const float* tc = a.chunk_tot + (size_t)h * s.n_chunks * kB;
-  float M = -INFINITY;
-  for (int c = lane; c < s.n_chunks; c += 32) M = fmaxf(M, mc[c * kB + r]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  double Z = 0.0;
-  for (int c = lane; c < s.n_chunks; c += 32) Z += (double)exp2f(mc[c * kB + r] - M) * (double)tc[c * kB + r];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, o);
-  float* w = a.row_w + (size_t)h * s.n_chunks * kB;
-  const double inv = 1.0 / (Z * kB);
-  for (int c = lane; c < s.n_chunks; c += 32) w[c * kB + r] = (float)((double)exp2f(mc[c * kB + r] - M) * inv);
-}
-
-// 2. Block masses, one warp per key block: p_v[kb] = sum_r w*(lo+hi). A row r whose split column
-//    is (t_last + r) mod 128 (t_last = n - 128 (N_b-1), 128 when n is a multiple of 128) meets
-//    slash blocks N_b-1-kb (lo) and N_b-2-kb (hi) when t_last + r >= 128, else N_b-2-kb (lo) and
-//    N_b-3-kb (hi) (CRISP §4, both directions). Every slot of ps_lo, ps_hi and ps_x is written
-//    once: by the key block that maps there, or with 0 by the block whose target lies below 0.
-constexpr int MASS_WARPS = 16;
-__global__ void __launch_bounds__(MASS_WARPS * 32) block_mass_kernel(const SelectArgs a) {
-  const Shape& s = a.s;
-  const int h = blockIdx.y, nb = s.nb;
-  const int kb = blockIdx.x * MASS_WARPS + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (kb >= nb) return;
-  const int t_last = s.n - (nb - 1) * kB;
-  const float2* p = a.part + ((size_t)h * nb + kb) * kB;
-  const float* wc = a.row_w + ((size_t)h * s.n_chunks + kb / kProxyChunk) * kB;
-  double loA = 0.0, hiA = 0.0, loB = 0.0, hiB = 0.0;
-#pragma unroll
-  for (int i = 0; i < kB / 32; ++i) {
-    const int r = lane + 32 * i;
-    const float2 v = p[r];
-    const double ww = wc[r];
-    if (t_last + r >= kB) {
-      loA += (double)v.x * ww;
-      hiA += (double)v.y * ww;
-    } else {
-      loB += (double)v.x * ww;
-      hiB += (double)v.y * ww;
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    loA += __shfl_xor_sync(0xffffffffu, loA, o);
-    hiA += __shfl_xor_sync(0xffffffffu, hiA, o);
-    loB += __shfl_xor_sync(0xffffffffu, loB, o);
-    hiB += __shfl_xor_sync(0xffffffffu, hiB, o);
-  }
-  if (lane == 0) {
-    const size_t base = (size_t)h * nb;
-    a.pv[base + kb] = (loA + hiA) + (loB + hiB);
-    a.ps_lo[base + nb - 1 - kb] = loA;
-    if (nb - 2 - kb >= 0) a.ps_hi[base + nb - 2 - kb] = hiA + loB;
-    else a.ps_hi[base + nb - 1] = 0.0;  // kb = N_b-1: the slot no block maps to
-    if (nb - 3 - kb >= 0) a.ps_x[base + nb - 3 - kb] = hiB;
-    else a.ps_x[base + (nb - 3 - kb == -1 ? nb - 2 : nb - 1)] = 0.0;  // kb = N_b-2, N_b-1
-  }
 }
 
 // Block-wide maximum and sum of doubles (all threads receive the result).
@@ -292,11 +224,12 @@ __device__ double median_inner(const double* p, int* sidx, int nb, int P2) {
   return med;
 }
 
-// 3. Per head: C_struct (or the JSD), route, noise floors, keep flags (+ top-up).
-__global__ void __launch_bounds__(THREADS) route_threshold_kernel(const SelectArgs a) {
+// 3. Per head: C_struct (or the JSD), route, noise floors, keep flags (+ top-up). Run by the
+//    last CTA of the head's block-mass kernel (every CTA of the head has written its masses).
+__device__ void route_head(const SelectArgs& a, int h) {
   extern __shared__ double dsm[];
   const Shape& s = a.s;
-  const int nb = s.nb, h = blockIdx.x, tid = threadIdx.x;
+  const int nb = s.nb, tid = threadIdx.x;
   double* pv = dsm;        // [nb]
   double* ps = dsm + nb;   // [nb]
   double* aux = dsm + 2 * nb;                  // [nb] doubles: a_bar, then sort indices
@@ -307,9 +240,11 @@ __global__ void __launch_bounds__(THREADS) route_threshold_kernel(const SelectAr
   __shared__ float qm[kD];
   __shared__ float qpart[THREADS / kD][kD];
   __shared__ int pos_min;
+  // written by the head's other CTAs: read through L2
   for (int i = tid; i < nb; i += THREADS) {
-    pv[i] = a.pv[(size_t)h * nb + i];
-    ps[i] = a.ps_lo[(size_t)h * nb + i] + a.ps_hi[(size_t)h * nb + i] + a.ps_x[(size_t)h * nb + i];
+    pv[i] = __ldcg(a.pv + (size_t)h * nb + i);
+    ps[i] = __ldcg(a.ps_lo + (size_t)h * nb + i) + __ldcg(a.ps_hi + (size_t)h * nb + i) +
+            __ldcg(a.ps_x + (size_t)h * nb + i);
   }
   __syncthreads();
 
@@ -322,7 +257,7 @@ __global__ void __launch_bounds__(THREADS) route_threshold_kernel(const SelectAr
   if (t_last != kB && nb >= 3) {
     const float* wr = a.row_w + ((size_t)h * s.n_chunks + (nb - 2) / kProxyChunk) * kB;
     double x = 0.0;
-    for (int r = tid; r < kB; r += THREADS) x += (double)a.rec_extra[(size_t)h * kB + r] * (double)wr[r];
+    for (int r = tid; r < kB; r += THREADS) x += (double)a.rec_extra[(size_t)h * kB + r] * (double)__ldcg(wr + r);
     C += block_sum(x, red);
   }
   double jsd = 0.0;
@@ -416,16 +351,102 @@ __global__ void __launch_bounds__(THREADS) route_threshold_kernel(const SelectAr
   }
 }
 
+// 1-2. One CTA per run of MASS_BLOCKS key blocks of a head:
+//   (a) per proxy row r: the global reference max M_r over the chunks, the normaliser Z_r, and
+//       for the CTA's chunks the weight w = exp2(m_chunk - M_r) / (Z_r * B) that turns a chunk's
+//       sums into column-mean mass (four threads per row, fp64 sums);
+//   (b) block masses, one warp per key block: p_v[kb] = sum_r w*(lo+hi). A row r whose split
+//       column is (t_last + r) mod 128 (t_last = n - 128 (N_b-1), 128 when n is a multiple of
+//       128) meets slash blocks N_b-1-kb (lo) and N_b-2-kb (hi) when t_last + r >= 128, else
+//       N_b-2-kb (lo) and N_b-3-kb (hi) (CRISP §4, both directions). Every slot of ps_lo, ps_hi
+//       and ps_x is written once: by the key block that maps there, or with 0 by the block whose
+//       target lies below 0;
+//   (c) the head's last CTA to finish routes the head (route_head).
+constexpr int MASS_BLOCKS = 64;                     // key blocks per CTA
+constexpr int MASS_CHUNKS = MASS_BLOCKS / kProxyChunk;
+__global__ void __launch_bounds__(THREADS) mass_route_kernel(const SelectArgs a) {
+  const Shape& s = a.s;
+  const int h = blockIdx.y, nb = s.nb, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int kb0 = blockIdx.x * MASS_BLOCKS;
+  const int c0 = kb0 / kProxyChunk, c1 = min(s.n_chunks, c0 + MASS_CHUNKS);
+  __shared__ float w_s[MASS_CHUNKS][kB];
+  {
+    const int r = tid >> 2, part = tid & 3;  // four threads per row, chunks part, part+4, ...
+    const float* mc = a.chunk_max + (size_t)h * s.n_chunks * kB;
+    const float* tc = a.chunk_tot + (size_t)h * s.n_chunks * kB;
+    float M = -INFINITY;
+    for (int c = part; c < s.n_chunks; c += 4) M = fmaxf(M, mc[c * kB + r]);
+    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 1));
+    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 2));
+    double Z = 0.0;
+    for (int c = part; c < s.n_chunks; c += 4) Z += (double)exp2f(mc[c * kB + r] - M) * (double)tc[c * kB + r];
+    Z += __shfl_xor_sync(0xffffffffu, Z, 1);
+    Z += __shfl_xor_sync(0xffffffffu, Z, 2);
+    const double inv = 1.0 / (Z * kB);
+    const int c = c0 + part;
+    if (c < c1) {
+      const float w = (float)((double)exp2f(mc[c * kB + r] - M) * inv);
+      w_s[part][r] = w;
+      a.row_w[((size_t)h * s.n_chunks + c) * kB + r] = w;
+    }
+  }
+  __syncthreads();
+  const int t_last = s.n - (nb - 1) * kB;
+  for (int kb = kb0 + warp; kb < min(nb, kb0 + MASS_BLOCKS); kb += NWARP) {
+    const float2* p = a.part + ((size_t)h * nb + kb) * kB;
+    const float* wc = w_s[kb / kProxyChunk - c0];
+    double loA = 0.0, hiA = 0.0, loB = 0.0, hiB = 0.0;
+    float2 v[kB / 32];
+#pragma unroll
+    for (int i = 0; i < kB / 32; ++i) v[i] = p[lane + 32 * i];
+#pragma unroll
+    for (int i = 0; i < kB / 32; ++i) {
+      const int r = lane + 32 * i;
+      const double ww = wc[r];
+      if (t_last + r >= kB) {
+        loA += (double)v[i].x * ww;
+        hiA += (double)v[i].y * ww;
+      } else {
+        loB += (double)v[i].x * ww;
+        hiB += (double)v[i].y * ww;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      loA += __shfl_xor_sync(0xffffffffu, loA, o);
+      hiA += __shfl_xor_sync(0xffffffffu, hiA, o);
+      loB += __shfl_xor_sync(0xffffffffu, loB, o);
+      hiB += __shfl_xor_sync(0xffffffffu, hiB, o);
+    }
+    if (lane == 0) {
+      const size_t base = (size_t)h * nb;
+      a.pv[base + kb] = (loA + hiA) + (loB + hiB);
+      a.ps_lo[base + nb - 1 - kb] = loA;
+      if (nb - 2 - kb >= 0) a.ps_hi[base + nb - 2 - kb] = hiA + loB;
+      else a.ps_hi[base + nb - 1] = 0.0;  // kb = N_b-1: the slot no block maps to
+      if (nb - 3 - kb >= 0) a.ps_x[base + nb - 3 - kb] = hiB;
+      else a.ps_x[base + (nb - 3 - kb == -1 ? nb - 2 : nb - 1)] = 0.0;  // kb = N_b-2, N_b-1
+    }
+  }
+  // the head's last CTA routes it (counter back to zero for the radix levels that reuse it)
+  __threadfence();
+  __syncthreads();
+  __shared__ int last;
+  if (tid == 0) last = atomicAdd(a.cut_done + h, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  if (tid == 0) a.cut_done[h] = 0;
+  route_head(a, h);
+}
+
 }  // namespace
 
 cudaError_t launch_route_threshold(const SelectArgs& a, cudaStream_t st) {
-  row_stats_kernel<<<dim3(kB / STAT_ROWS, a.s.h_q), STAT_ROWS * 32, 0, st>>>(a);
-  block_mass_kernel<<<dim3((a.s.nb + MASS_WARPS - 1) / MASS_WARPS, a.s.h_q), MASS_WARPS * 32, 0, st>>>(a);
   const size_t smem = (size_t)3 * a.s.nb * sizeof(double);  // p_v, p_s, and a_bar / sort indices
-  cudaError_t e = cudaFuncSetAttribute(route_threshold_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(mass_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  route_threshold_kernel<<<a.s.h_q, THREADS, smem, st>>>(a);
+  mass_route_kernel<<<dim3((a.s.nb + MASS_BLOCKS - 1) / MASS_BLOCKS, a.s.h_q), THREADS, smem, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -122,7 +122,7 @@ def compare_selection(index, sels: dict, nb: int, log: list | None = None, name:
         else:
             for qb in range(nb):
                 assert gl[qb] == ol[qb].tolist()
-    rec.update(stats)
+    rec["counts"] = dict(stats)
     if log is not None and (stats["vs_tie_blocks"] or stats["pe_differing"]):
         log.append(f"ties: {stats}")
     return stats

@@ -4,9 +4,9 @@ Some callers cannot allocate device memory: a serving engine whose memory manage
 device byte, or a latency-critical path that cannot afford the device synchronisation an
 allocation implies. They call crisp_select_noalloc, which keeps its scratch in a fixed array
 inside the library instead of a caller-provided workspace. Its index must equal crisp_select's
-exactly, on two calls in a row (the array keeps the previous call's contents, so a second call
-over different inputs checks that nothing stale leaks through), and shapes that need more
-scratch than the array holds must be refused before anything is launched.
+exactly on consecutive calls over different inputs of the same shape (the array keeps the
+previous call's contents, so nothing stale may leak through), and shapes that need more scratch
+than the array holds must be refused before anything is launched.
 """
 import ctypes
 
@@ -48,22 +48,30 @@ def _same_index(a, b, nb):
 
 
 def test_noalloc_select_matches_select_on_consecutive_calls():
+    """Per shape: planted inputs, then different inputs of the same shape (all heads diffuse, so
+    every head takes the other route and its scratch regions hold other values), then the
+    planted inputs again; each call must equal crisp_select on its own inputs."""
     dev = torch.device("cuda:0")
     f = _entry()
     cases = [(W.WORKLOADS["llama8b_32k"].scaled(4096), crisp.Params()),
              (W.WORKLOADS["qwen7b_128k"].scaled(2048), crisp.Params(min_blocks=4))]
     for w, params in cases:
         q, k, _, _ = W.generate(w)
-        q, k = q.to(dev), k.to(dev)
-        ref = crisp.select(q, k, params, debug=True)
+        q2, k2, _ = W.random_qkv(w.h_q, w.h_kv, w.n, seed=w.n + 1)
+        inputs = [(q.to(dev), k.to(dev)), (q2.to(dev), k2.to(dev))]
+        refs = []
+        for qq, kk in inputs:
+            refs.append(crisp.select(qq, kk, params, debug=True))
         torch.cuda.synchronize()
-        for _ in range(2):
+        assert not torch.equal(refs[0].route, refs[1].route)
+        for which in (0, 1, 0):
+            qq, kk = inputs[which]
             got = crisp.Index.empty(w.h_q, w.n, dev, debug=True)
             status = torch.zeros(1, dtype=torch.int32, device=dev)
-            assert _call(f, q, k, params, got, status) == 0
+            assert _call(f, qq, kk, params, got, status) == 0
             torch.cuda.synchronize()
             assert int(status.item()) == 0
-            _same_index(ref, got, w.n // 128)
+            _same_index(refs[which], got, w.n // 128)
 
 
 def test_noalloc_select_refuses_shapes_beyond_its_array():
