@@ -39,8 +39,8 @@ struct CutState {
 
 struct Workspace {
   size_t status, trace, part, chunk_max, chunk_tot, row_w, pv, ps_lo, ps_hi, ps_x, rec_extra, kbar, kparts, qparts,
-      pbuf, hist_cnt, hist_mass, cut, cut_done, keep_v, keep_s, cnt, eqcnt, eqbase, selmask, idx_route, idx_c,
-      idx_row_ptr, idx_cols, total;
+      pbuf, hist_cnt, hist_mass, cut, cut_done, anchor_cnt, hint, hint_ready, pooled_cnt, keep_v, keep_s, cnt,
+      eqcnt, eqbase, selmask, idx_route, idx_c, idx_row_ptr, idx_cols, total;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -59,24 +59,29 @@ inline Workspace workspace_layout(const Shape& s) {
   const size_t hq = s.h_q, nb = s.nb, ch = s.n_chunks;
   w.status = take(256);
   w.trace = take((size_t)256 * 2 * 8 * 8);
-  w.part = take(hq * nb * kB * 8);
-  w.chunk_max = take(hq * ch * kB * 4);
-  w.chunk_tot = take(hq * ch * kB * 4);
-  w.row_w = take(hq * ch * kB * 4);
+  // the proxy pass keeps one reference per (chunk, 64-column half) "segment" and proxy row
+  w.part = take(hq * nb * 2 * kB * 8);
+  w.chunk_max = take(hq * ch * 2 * kB * 4);
+  w.chunk_tot = take(hq * ch * 2 * kB * 4);
+  w.row_w = take(hq * ch * 2 * kB * 4);
   w.pv = take(hq * nb * 8);
   w.ps_lo = take(hq * nb * 8);
   w.ps_hi = take(hq * nb * 8);
   w.ps_x = take(hq * nb * 8);
-  w.rec_extra = take(hq * kB * 4);
+  w.rec_extra = take(hq * 2 * kB * 4);
   w.kbar = take((size_t)s.h_kv * nb * kD * 4);
   w.kparts = take((size_t)s.h_kv * 3 * nb * kD * 2);
   w.qparts = take(hq * 3 * nb * kD * 2);
   w.pbuf = take(hq * (size_t)s.cap * 4);
-  // hist_cnt .. cut_done are contiguous: one memset clears them at the start of a selection
+  // hist_cnt .. pooled_cnt are contiguous: one memset clears them at the start of a selection
   w.hist_cnt = take(hq * kHistBins * 4);
   w.hist_mass = take(hq * kHistBins * 8);
   w.cut = take(hq * sizeof(CutState));
   w.cut_done = take(hq * 4);
+  w.anchor_cnt = take(hq * 4);
+  w.hint = take(hq * 4);
+  w.hint_ready = take(hq * 4);
+  w.pooled_cnt = take(hq * 4);
   w.keep_v = take(hq * nb);
   w.keep_s = take(hq * nb);
   w.cnt = take(hq * nb * 4);
@@ -102,15 +107,15 @@ struct SelectArgs {
   int floor_rule;  // 0: mean floor; 1: median floor
   int* status;
   unsigned long long* trace;
-  float2* part;
-  float* chunk_max;
-  float* chunk_tot;
-  float* row_w;
+  float2* part;        // [h_q][N_b][half][128]: per key block, half and proxy row (lower, upper) sums
+  float* chunk_max;    // [h_q][chunk][half][128]: the segment's reference (log2 units)
+  float* chunk_tot;    // ... and its total against that reference
+  float* row_w;        // ... and the weight that turns its sums into column-mean mass
   double* pv;      // vertical block masses
   double* ps_lo;   // slash block masses from the keys at or below each row's diagonal offset
   double* ps_hi;   // ... and from the keys above it
   double* ps_x;    // ... and (n not a multiple of 128) the next offset block down
-  float* rec_extra;  // per proxy row: recency-window mass inside block N_b-2 (n not a multiple of 128)
+  float* rec_extra;  // [h_q][half][128]: recency-window mass inside block N_b-2 (n not a multiple of 128)
   float* kbar;                  // K_bar fp32 [h_kv][N_b][128]
   __nv_bfloat16* kparts;        // K_bar as three bf16 terms [h_kv][3][N_b][128] (sum exact)
   __nv_bfloat16* qparts;        // Q_bar of PE heads, likewise [h_q][3][N_b][128]
@@ -119,6 +124,13 @@ struct SelectArgs {
   unsigned long long* hist_mass;  // fixed point, 2^-40 units
   CutState* cut;
   uint32_t* cut_done;           // per head: CTAs of the current radix level that finished
+  // Q_bar pooling during the proxy pass (see proxy_pass.cu): per head pair, anchor chunks done;
+  // per head, the early Pooled-Estimation hint, its ready flag, and the 16-block runs pooled
+  uint32_t* anchor_cnt;
+  uint32_t* hint;
+  uint32_t* hint_ready;
+  uint32_t* pooled_cnt;
+  int proxy_ctas;               // CTAs of the proxy pass that run proxy items (the rest pool Q_bar)
   uint8_t* keep_v;
   uint8_t* keep_s;
   int* cnt;

@@ -5,7 +5,8 @@
 // For every head routed to PE:
 //   qbar_kernel     Q_bar[qb] = mean of the block's query rows (fp32; 128, or fewer in a partial
 //                   last block), read once from HBM, stored as three bf16 terms whose sum is the
-//                   fp32 value exactly (hi, mid, lo);
+//                   fp32 value exactly (hi, mid, lo) — for the PE heads the proxy pass did not
+//                   already pool while it ran;
 //   scores_kernel   logits Q_bar[qb] . K_bar[kb] / sqrt(d) for kb <= qb, one 128x128 tile per
 //                   CTA on the tensor cores: the six products hi.hi + hi.mid + mid.hi + hi.lo +
 //                   mid.mid + lo.hi of the split operands accumulate in fp32 in TMEM (the terms
@@ -43,6 +44,8 @@ __global__ void __launch_bounds__(128) qbar_kernel(const SelectArgs a) {
   const int qb = blockIdx.x, h = blockIdx.y;
   if (!is_pe(a, h)) return;
   const Shape& s = a.s;
+  // heads the proxy pass pooled already (every run of 16 query blocks counted)
+  if (a.pooled_cnt[h] == (uint32_t)((s.nb + kProxyChunk - 1) / kProxyChunk)) return;
   const int t = threadIdx.x, c16 = t & 15, rg = t >> 4;
   const __nv_bfloat16* base = a.q + ((size_t)h * s.ld + (size_t)qb * kB) * kD + c16 * 8;
   float acc[8];
@@ -211,33 +214,47 @@ __global__ void __launch_bounds__(SC_THREADS) scores_kernel(const __grid_constan
 }
 
 // ------------------------------------------------------------------------ histograms, select
-// Histogram masses are fixed point (2^-40 units, rounded): integer atomics are exact and
-// order-independent, and N_b * 2^40 stays far below 2^64.
+// Histogram masses are fixed point (2^-40 units, rounded to nearest, ties to even): integer
+// atomics are exact and order-independent, and N_b * 2^40 stays far below 2^64. For p >= 0 with
+// biased exponent e and 24-bit significand s, p * 2^40 = s * 2^(e - 110): a shift of s, rounded
+// when it runs right, all in integer arithmetic.
 __device__ __forceinline__ unsigned long long to_fixed(float p) {
-  return __double2ull_rn((double)p * kMassUnit);
+  const uint32_t bits = __float_as_uint(p);
+  const int e = (int)(bits >> 23);
+  if (e == 0) return 0ull;  // zero, or below 2^-126: rounds to 0
+  const unsigned long long sig = (bits & 0x7fffffu) | 0x800000u;
+  const int sh = e - 110;
+  if (sh >= 0) return sig << sh;
+  const int k = -sh;
+  if (k > 25) return 0ull;
+  const unsigned long long q = sig >> k, rem = sig & ((1ull << k) - 1ull), half = 1ull << (k - 1);
+  return q + ((rem > half || (rem == half && (q & 1ull))) ? 1ull : 0ull);
 }
 
-// Warp-aggregated update for rows whose values mostly share a bin: lanes with the same bin are
-// summed first, one shared atomic per distinct bin. All lanes must call it.
-__device__ __forceinline__ void warp_hist_add(uint32_t* scnt, unsigned long long* smass, bool valid, uint32_t bin,
-                                              unsigned long long fx) {
-  const int lane = threadIdx.x & 31;
-  unsigned todo = __ballot_sync(0xffffffffu, valid);
-  while (todo) {
-    const int leader = __ffs(todo) - 1;
-    const uint32_t lb = __shfl_sync(0xffffffffu, bin, leader);
-    const bool mine = ((todo >> lane) & 1u) && bin == lb;
-    const unsigned grp = __ballot_sync(0xffffffffu, mine);
-    unsigned long long v = mine ? fx : 0ull;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == leader) {
-      atomicAdd(&scnt[lb], (uint32_t)__popc(grp));
-      atomicAdd(&smass[lb], v);
+// Per-lane run of histogram updates: consecutive entries of one lane that fall in the same bin are
+// counted and summed in registers and go to shared memory (two atomics) only when the bin
+// changes. A pooled row's probabilities mostly share a few bins, so a lane flushes a few times
+// per row.
+struct BinRun {
+  uint32_t bin = 0xffffffffu, cnt = 0u;
+  unsigned long long mass = 0ull;
+  __device__ __forceinline__ void add(uint32_t* scnt, unsigned long long* smass, uint32_t b, unsigned long long fx) {
+    if (b != bin) {
+      flush(scnt, smass);
+      bin = b;
     }
-    todo &= ~grp;
+    ++cnt;
+    mass += fx;
   }
-}
+  __device__ __forceinline__ void flush(uint32_t* scnt, unsigned long long* smass) {
+    if (cnt) {
+      atomicAdd(&scnt[bin], cnt);
+      atomicAdd(&smass[bin], mass);
+    }
+    cnt = 0u;
+    mass = 0ull;
+  }
+};
 
 // Adds a CTA's shared histogram to the head's global one, then reports whether this CTA is the
 // last of the head's `ctas` to finish (that CTA then sees every CTA's counts).
@@ -378,7 +395,7 @@ __device__ void select_bin(const SelectArgs& a, int h, int level) {
 // stays in registers (32 per lane, all loads in flight at once); longer rows take three passes
 // over memory. Exponentials use the exp2 unit on log2(e)-scaled logits.
 constexpr int ROWS_PER_CTA = 8;
-__global__ void __launch_bounds__(ROWS_PER_CTA * 32) rowsoft_kernel(const SelectArgs a) {
+__global__ void __launch_bounds__(ROWS_PER_CTA * 32, 4) rowsoft_kernel(const SelectArgs a) {
   const int h = blockIdx.y;
   if (!is_pe(a, h)) return;
   const Shape& s = a.s;
@@ -419,16 +436,17 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32) rowsoft_kernel(const Select
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
       const float inv = 1.f / z;
+      BinRun run;
 #pragma unroll
       for (int u = 0; u < 32; ++u) {
-        if (u * 32 < L) {
-          const int i = u * 32 + lane;
-          const bool valid = i < L;
+        const int i = u * 32 + lane;
+        if (u * 32 < L && i < L) {
           const float p = x[u] * inv;
-          if (valid) row[i] = p;
-          warp_hist_add(scnt, smass, valid, __float_as_uint(p) >> 20, to_fixed(p));
+          row[i] = p;
+          run.add(scnt, smass, __float_as_uint(p) >> 20, to_fixed(p));
         }
       }
+      run.flush(scnt, smass);
     } else {
       float mx = -INFINITY;
       for (int base = 0; base < L; base += 256) {
@@ -464,6 +482,7 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32) rowsoft_kernel(const Select
       for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
       const float inv = 1.f / z;
       __syncwarp();
+      BinRun run;
       for (int base = 0; base < L; base += 256) {
         float e[8];
 #pragma unroll
@@ -474,12 +493,14 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32) rowsoft_kernel(const Select
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const int i = base + 32 * u + lane;
-          const bool valid = i < L;
-          const float p = e[u] * inv;
-          if (valid) row[i] = p;
-          warp_hist_add(scnt, smass, valid, __float_as_uint(p) >> 20, to_fixed(p));
+          if (i < L) {
+            const float p = e[u] * inv;
+            row[i] = p;
+            run.add(scnt, smass, __float_as_uint(p) >> 20, to_fixed(p));
+          }
         }
       }
+      run.flush(scnt, smass);
     }
   }
   __syncthreads();

@@ -7,18 +7,21 @@
 // grid is persistent (one CTA per SM): CTA c takes a contiguous run of the items listed pair by
 // pair, so a CTA's items mostly share their Q tiles, and the barrier rings run on from one item
 // to the next.
-//   warp 8      TMA producer: the two Q tiles whenever the pair changes (after the MMAs that read
+//   warp 16     TMA producer: the two Q tiles whenever the pair changes (after the MMAs that read
 //               the old ones), then the chunks' K blocks through a 3-stage ring;
-//   warp 9      one thread issues S_t = Q_t K_blk^T (128x128x128, bf16 -> fp32) into a
+//   warp 17     one thread issues S_t = Q_t K_blk^T (128x128x128, bf16 -> fp32) into a
 //               double-buffered TMEM tile per head;
-//   warps 0-7   softmax, one warpgroup per head, one proxy row per thread: read the S row from
-//               TMEM 32 columns at a time (the next load in flight while the current columns are
-//               exponentiated), mask the keys the causal limit cuts (key j visible to row r iff
-//               j <= n-B+r), and accumulate exp2(x - m) against a lagging row reference m (set
-//               by the chunk's first block, moved only when a block's sum would leave [0, 2^64])
-//               into two sums per key block: keys at or below the row's diagonal offset (t <= r)
-//               and above it (t > r);
-//   warps 10-11 sum rows of each K block into the mean-pooled key K_bar of the PE path; the
+//   warps 0-15  softmax: per head 8 warps, two per TMEM lane quarter, each thread one proxy row
+//               and one 64-column half of the S block (four exponentiating warps per
+//               sub-partition keep the exp2 unit fed): read its columns from TMEM 32 at a time
+//               (the next load in flight while the current columns are exponentiated), mask the
+//               keys the causal limit cuts (key j visible to row r iff j <= n-B+r), and
+//               accumulate exp2(x - m) against a lagging reference m of its own (set by its first
+//               block of the chunk, moved only when a block's sum would leave [0, 2^64]) into two
+//               sums per key block: keys at or below the row's diagonal offset (t <= r) and above
+//               it (t > r). Each (chunk, half) is a segment with its own reference; the sums go
+//               straight to global memory and the routing kernel weighs the segments;
+//   warps 18-19 sum rows of each K block into the mean-pooled key K_bar of the PE path; the
 //               items of one group share the 16 column chunks between them.
 // A key at offset t of block kb seen by proxy row r lies on diagonal offset (N_b-1-kb)*B + (r-t),
 // so the first sum belongs to slash block N_b-1-kb and the second to N_b-2-kb; their total is
@@ -33,18 +36,32 @@ namespace crisp {
 namespace {
 
 constexpr int NS = 3;
-constexpr int THREADS = 384;
-constexpr int PRODUCER_WARP = 8;
-constexpr int MMA_WARP = 9;
-constexpr int POOL_WARP = 10;   // and 11: two warps share the pooling
+constexpr int SOFTMAX_WARPS = 16;
+constexpr int PRODUCER_WARP = 16;
+constexpr int MMA_WARP = 17;
+constexpr int POOL_WARP = 18;   // and 19: two warps share the pooling
+constexpr int THREADS = 640;
 constexpr uint32_t TILE_BYTES = kB * kD * 2;
 constexpr uint32_t HALF_BYTES = TILE_BYTES / 2;
 constexpr float kScaleLog2 = 0.12751743074380045f;  // log2(e) / sqrt(128)
 
+constexpr int POOL_STAGES = 5;  // Q blocks in flight in a pooling CTA (over the q and k buffers)
+// Share of the SMs that pool Q_bar during the proxy pass (numerator / denominator).
+#ifndef CRISP_POOL_SHARE_NUM
+#define CRISP_POOL_SHARE_NUM 16
+#endif
+constexpr int kPoolShareNum = CRISP_POOL_SHARE_NUM;
+constexpr int kPoolShareDen = 100;
+
 struct __align__(1024) ProxySmem {
   __nv_bfloat16 q[2][kB * kD];  // two 128-byte-swizzled halves [128 rows][64 cols] per tile
   __nv_bfloat16 k[NS][kB * kD];
-  float2 part[2][kProxyChunk][kB];  // per tile, block and row: (lower, upper) sums
+  float red[2][32][kD];         // pooling CTAs: per-row-group partial sums of a Q block
+  uint64_t pool_full[POOL_STAGES];
+  uint64_t pool_empty[POOL_STAGES];
+  int stage_info[POOL_STAGES];  // head * 65536 + query block of the stage, or -1: no more
+  float hint_part[2][4];
+  int anchor_last;
   uint64_t q_full;
   uint64_t q_empty;
   uint64_t k_full[NS];
@@ -75,13 +92,13 @@ __device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&r)[32]) {
       : "memory");
 }
 
-// Item `it` of the pair-major list: (pair, chunk) and what follows from them.
+// Item (pair, chunk) and what follows from it.
 struct Item {
   int pair, chunk, kv, pig, h0, ntiles, kb0, nblk;
-  __device__ __forceinline__ Item(const Shape& s, int it) {
+  __device__ __forceinline__ Item(const Shape& s, int pair_, int chunk_) {
     const int ppg = (s.G + 1) / 2;
-    pair = it / s.n_chunks;
-    chunk = it % s.n_chunks;
+    pair = pair_;
+    chunk = chunk_;
     kv = pair / ppg;
     pig = pair % ppg;
     h0 = kv * s.G + 2 * pig;
@@ -91,20 +108,65 @@ struct Item {
   }
 };
 
-// One block of one row, the common case (n a multiple of 128, not the last block): S read 32
-// columns at a time (the next load in flight while these are exponentiated), and the row's sums
-// below/above its diagonal column r (warp `grp` holds rows 32grp..32grp+31, so columns
-// of chunk c < grp are all below, c > grp all above, and chunk grp splits at the lane).
-__device__ __forceinline__ void block_sums_fast(uint32_t sbase, float nm, int grp, int lane, float& lo, float& hi) {
+// Which items a proxy CTA runs. The items are the (head pair, chunk) pairs; CTA c runs a
+// contiguous share of them. With early pooling ("anchored"), CTA c < A first runs anchor item c
+// — the chunks holding a pair's sink block (chunk 0) and last block (chunk n_chunks-1), which
+// bound the pair's C_struct from above — and then its share of the other items, listed pair by
+// pair; otherwise its share of the pair-major list.
+struct Sched {
+  int I, A, apc, nac, n_proxy, n_chunks;
+  bool anchored;
+  __device__ __forceinline__ Sched(const Shape& s, int n_proxy_, bool anchored_) {
+    const int pairs = s.h_kv * ((s.G + 1) / 2);
+    n_chunks = s.n_chunks;
+    I = pairs * n_chunks;
+    apc = min(2, n_chunks);
+    A = pairs * apc;
+    nac = n_chunks - apc;
+    n_proxy = n_proxy_;
+    anchored = anchored_;
+  }
+  __device__ __forceinline__ int count(int c) const {
+    return (int)(((long long)(c + 1) * I) / n_proxy - ((long long)c * I) / n_proxy);
+  }
+  __device__ __forceinline__ bool is_anchor(int c, int k) const { return anchored && c < A && k == 0; }
+  __device__ __forceinline__ void at(int c, int k, int& pair, int& chunk) const {
+    const long long start = ((long long)c * I) / n_proxy;
+    if (!anchored) {
+      const long long it = start + k;
+      pair = (int)(it / n_chunks);
+      chunk = (int)(it % n_chunks);
+    } else if (c < A && k == 0) {
+      pair = c / apc;
+      chunk = (c % apc == 0) ? n_chunks - 1 : 0;
+    } else {
+      const long long x = start - min(c, A) + k - (c < A ? 1 : 0);  // index among the other items
+      pair = (int)(x / nac);
+      chunk = 1 + (int)(x % nac);
+    }
+  }
+};
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// One block of one row and one 64-column half, the common case (n a multiple of 128, not the
+// last block): S read 32 columns at a time (the next load in flight while these are
+// exponentiated), and the sums below/above the row's diagonal column r (warp `grp` holds rows
+// 32grp..32grp+31, so columns of 32-column chunk c < grp are all below, c > grp all above, and
+// chunk grp splits at the lane).
+__device__ __forceinline__ void block_sums_fast(uint32_t sbase, float nm, int grp, int lane, int half, float& lo,
+                                                float& hi) {
   uint32_t v[2][32];
   lo = 0.f;
   hi = 0.f;
   tmem_ld32(sbase, v[0]);
   tmem_ld_wait_regs(v[0]);
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    uint32_t(&x)[32] = v[c & 1];
-    if (c < 3) tmem_ld32(sbase + (c + 1) * 32, v[(c + 1) & 1]);
+  for (int c = 0; c < 2; ++c) {
+    uint32_t(&x)[32] = v[c];
+    if (c == 0) tmem_ld32(sbase + 32, v[1]);
     float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int q = 0; q < 32; ++q) {
@@ -113,9 +175,10 @@ __device__ __forceinline__ void block_sums_fast(uint32_t sbase, float nm, int gr
       s4[q & 3] += e;
     }
     const float sc = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-    if (c < grp) {
+    const int cc = 2 * half + c;  // chunk index within the 128 columns
+    if (cc < grp) {
       lo += sc;
-    } else if (c > grp) {
+    } else if (cc > grp) {
       hi += sc;
     } else {
       float l2[2] = {0.f, 0.f}, h2[2] = {0.f, 0.f};
@@ -127,35 +190,220 @@ __device__ __forceinline__ void block_sums_fast(uint32_t sbase, float nm, int gr
       lo += l2[0] + l2[1];
       hi += h2[0] + h2[1];
     }
-    if (c < 3) tmem_ld_wait_regs(v[(c + 1) & 1]);
+    if (c == 0) tmem_ld_wait_regs(v[1]);
   }
 }
 
-// Largest logit of the row in this block (after the causal mask), scaled to log2 units.
-__device__ __forceinline__ float block_max_scaled(uint32_t sbase, int lim, bool edge) {
+// Largest logit of the row in one 64-column half of this block (after the causal mask; col0 is
+// the half's first column), scaled to log2 units.
+__device__ __forceinline__ float block_max_scaled(uint32_t sbase, int col0, int lim, bool edge) {
   uint32_t v[2][32];
   float mx = -INFINITY;
+  tmem_ld32(sbase, v[0]);
+  tmem_ld32(sbase + 32, v[1]);
+  tmem_ld_wait_regs(v[0]);
+  tmem_ld_wait_regs(v[1]);
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    tmem_ld32(sbase + h * 64, v[0]);
-    tmem_ld32(sbase + h * 64 + 32, v[1]);
-    tmem_ld_wait_regs(v[0]);
-    tmem_ld_wait_regs(v[1]);
+  for (int c = 0; c < 2; ++c)
+#pragma unroll
+    for (int q = 0; q < 32; q += 2) {
+      float a = __uint_as_float(v[c][q]), b = __uint_as_float(v[c][q + 1]);
+      if (edge) {
+        if (col0 + c * 32 + q > lim) a = -INFINITY;
+        if (col0 + c * 32 + q + 1 > lim) b = -INFINITY;
+      }
+      float m3;
+      asm("max.f32 %0, %1, %2, %3;" : "=f"(m3) : "f"(mx), "f"(a), "f"(b));
+      mx = m3;
+    }
+  return mx * kScaleLog2;
+}
+
+// End of an anchor item (run by all 16 softmax warps): the CTA that completes the second anchor
+// chunk of a head pair computes, for each of the pair's heads, an upper bound of its C_struct from
+// the two anchor chunks alone — the mass of the first and last 128 keys over the mass of the
+// anchor chunks' keys, whose total can only grow with the other chunks — and publishes
+// hint[h] = 1 (Pooled-Estimation for sure, up to rounding) when the bound is below tau_proxy.
+// Pooling CTAs start on Q_bar of hinted heads while the other chunks run. The hint only decides
+// when Q_bar is pooled, never a route.
+__device__ void anchor_done(ProxySmem& sm, const SelectArgs& a, const Item& w, int apc, int t, int half, int grp,
+                            int lane) {
+  const Shape& s = a.s;
+  __threadfence();  // this thread's sums and segment statistics, before the count
+  named_bar_sync(1, SOFTMAX_WARPS * 32);
+  if (threadIdx.x == 0) {
+    const bool aborted = *reinterpret_cast<volatile int*>(&sm.abort) != 0;
+    sm.anchor_last = (!aborted && atomicAdd(a.anchor_cnt + w.pair, 1u) == (unsigned)(apc - 1)) ? 1 : 0;
+  }
+  named_bar_sync(1, SOFTMAX_WARPS * 32);
+  if (!sm.anchor_last) return;
+  __threadfence();  // the other anchor's writes are visible
+  const int nb = s.nb, nch = s.n_chunks, last = nch - 1;
+  if (half == 0 && t < w.ntiles) {
+    const int h = w.h0 + t, r = grp * 32 + lane;
+    // segments (chunk, half) of chunks 0 and last: reference and total
+    float m[2][2], tot[2][2];
 #pragma unroll
     for (int c = 0; c < 2; ++c)
 #pragma unroll
-      for (int q = 0; q < 32; q += 2) {
-        float a = __uint_as_float(v[c][q]), b = __uint_as_float(v[c][q + 1]);
-        if (edge) {
-          if (h * 64 + c * 32 + q > lim) a = -INFINITY;
-          if (h * 64 + c * 32 + q + 1 > lim) b = -INFINITY;
-        }
-        float m3;
-        asm("max.f32 %0, %1, %2, %3;" : "=f"(m3) : "f"(mx), "f"(a), "f"(b));
-        mx = m3;
+      for (int hf = 0; hf < 2; ++hf) {
+        const int ch = c ? last : 0;
+        const size_t ci = (((size_t)h * nch + ch) * 2 + hf) * kB + r;
+        m[c][hf] = __ldcg(a.chunk_max + ci);
+        tot[c][hf] = (c == 1 && last == 0) ? 0.f : __ldcg(a.chunk_tot + ci);  // one chunk: count once
       }
+    float M = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) M = fmaxf(M, m[c][hf]);
+    float Z = 0.f, A = 0.f;
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) Z += tot[c][hf] * exp2f(m[c][hf] - M);
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const float2 p0 = __ldcg(a.part + ((size_t)h * nb * 2 + hf) * kB + r);  // block 0
+      A += (p0.x + p0.y) * exp2f(m[0][hf] - M);
+      if (nb > 1) {
+        const float2 pl = __ldcg(a.part + (((size_t)h * nb + nb - 1) * 2 + hf) * kB + r);
+        A += (pl.x + pl.y) * exp2f(m[1][hf] - M);
+      }
+      if (s.n % kB != 0 && nb >= 3) {
+        // the last 128 keys reach into block N_b-2 (its columns from t_last on), which lies in
+        // the last chunk or in chunk 0
+        const int cb = (nb - 2) / kProxyChunk;
+        if (cb == last || cb == 0)
+          A += __ldcg(a.rec_extra + ((size_t)h * 2 + hf) * kB + r) * exp2f(m[cb == last ? 1 : 0][hf] - M);
+      }
+    }
+    float c_row = Z > 0.f ? A / Z : 1.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c_row += __shfl_xor_sync(0xffffffffu, c_row, o);
+    if (lane == 0) sm.hint_part[t][grp] = c_row;
   }
-  return mx * kScaleLog2;
+  named_bar_sync(1, SOFTMAX_WARPS * 32);
+  if (threadIdx.x < w.ntiles) {
+    const int t2 = threadIdx.x, h = w.h0 + t2;
+    const float c_bound = (sm.hint_part[t2][0] + sm.hint_part[t2][1] + sm.hint_part[t2][2] + sm.hint_part[t2][3]) *
+                          (1.f / kB);
+    a.hint[h] = (a.route_rule == 0 && c_bound < a.tau) ? 1u : 0u;
+    __threadfence();
+    atomicExch(a.hint_ready + h, 1u);
+  }
+}
+
+// Q_bar pooling CTAs: pooling item i = (head, run of 16 query blocks), CTA p of P taking items
+// p, p+P, ... A producer thread waits (bounded) for the head's hint and, for a hinted head, loads
+// the run's Q blocks by TMA through POOL_STAGES stages laid over the q and k buffers; the 16
+// softmax-sized warps sum each block's rows (32 row groups of 4 rows, one 16-byte chunk of 8
+// columns per thread, then the 32 partial sums per column), take the mean and store it as three
+// bf16 terms, and count the run in pooled_cnt[head]. A head whose hint never came, or came 0, is
+// left to the Q_bar kernel after routing.
+constexpr unsigned long long kHintWaitNs = 4000000ull;  // 4 ms
+__device__ void pool_q_blocks(ProxySmem& sm, const CUtensorMap& q_map, const SelectArgs& a, int p, int P, int warp,
+                              int lane) {
+  const Shape& s = a.s;
+  const int ipr = (s.nb + kProxyChunk - 1) / kProxyChunk;  // runs of 16 query blocks per head
+  const int n_pool_items = s.h_q * ipr;
+  uint8_t* stage0 = reinterpret_cast<uint8_t*>(&sm.q[0][0]);
+  if (warp == PRODUCER_WARP) {
+    if (lane == 0) {
+      tma_prefetch_desc(&q_map);
+      int st = 0, given_up = -1;  // a head whose hint did not come in time is not waited for again
+      for (int pi = p; pi < n_pool_items; pi += P) {
+        const int h = pi / ipr, run = pi % ipr;
+        if (h == given_up) continue;
+        volatile uint32_t* ready = a.hint_ready + h;
+        const unsigned long long t0 = global_ns();
+        bool have = true;
+        while (*ready == 0u) {
+          if (global_ns() - t0 > kHintWaitNs || *reinterpret_cast<volatile int*>(&sm.abort)) {
+            have = false;
+            given_up = h;
+            break;
+          }
+          __nanosleep(256);
+        }
+        if (!have || *reinterpret_cast<volatile uint32_t*>(a.hint + h) == 0u) continue;
+        for (int qb = run * kProxyChunk; qb < min(s.nb, (run + 1) * kProxyChunk); ++qb, ++st) {
+          const int sg = st % POOL_STAGES;
+          if (!mbar_wait(&sm.pool_empty[sg], ((st / POOL_STAGES) & 1) ^ 1, nullptr)) {
+            fail(sm, a.status);
+            break;
+          }
+          sm.stage_info[sg] = h * 65536 + qb;
+          uint8_t* dst = stage0 + (size_t)sg * TILE_BYTES;
+          mbar_arrive_expect_tx(&sm.pool_full[sg], TILE_BYTES);
+          tma_load_3d(&q_map, &sm.pool_full[sg], dst, 0, qb * kB, h);
+          tma_load_3d(&q_map, &sm.pool_full[sg], dst + HALF_BYTES, 64, qb * kB, h);
+        }
+      }
+      // end marker: a plain arrival completes the stage's phase with no bytes
+      const int sg = st % POOL_STAGES;
+      if (mbar_wait(&sm.pool_empty[sg], ((st / POOL_STAGES) & 1) ^ 1, nullptr)) {
+        sm.stage_info[sg] = -1;
+        mbar_arrive(&sm.pool_full[sg]);
+      } else {
+        fail(sm, a.status);
+      }
+    }
+    __syncwarp();
+  } else if (warp < SOFTMAX_WARPS) {
+    const int tid = threadIdx.x;  // 0..511
+    const int cc = tid & 15, rg = tid >> 4;  // 8-column chunk, group of 4 rows
+    const int half = cc >> 3, ch = cc & 7;
+    for (int st = 0;; ++st) {
+      const int sg = st % POOL_STAGES;
+      if (!warp_wait(&sm.pool_full[sg], (st / POOL_STAGES) & 1, &sm.abort)) {
+        fail(sm, a.status);
+        break;
+      }
+      const int info = sm.stage_info[sg];
+      if (info < 0) break;
+      const int h = info >> 16, qb = info & 0xffff;
+      const uint8_t* base = stage0 + (size_t)sg * TILE_BYTES + half * HALF_BYTES;
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      uint4 u[4];
+#pragma unroll
+      for (int x = 0; x < 4; ++x) u[x] = *reinterpret_cast<const uint4*>(base + sw128_offset(rg * 4 + x, ch));
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&u[x]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __bfloat1622float2(p2[i]);
+          acc[2 * i] += f.x;
+          acc[2 * i + 1] += f.y;
+        }
+      }
+      float* red = &sm.red[st & 1][0][0];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) red[rg * kD + cc * 8 + i] = acc[i];
+      named_bar_sync(2, SOFTMAX_WARPS * 32);
+      if (tid == 0) mbar_arrive(&sm.pool_empty[sg]);  // every thread has read the stage
+      if (tid < kD) {
+        float v = 0.f;
+#pragma unroll 8
+        for (int g = 0; g < 32; ++g) v += red[g * kD + tid];
+        const int rows = min(kB, s.n - qb * kB);  // a partial last block has fewer rows
+        v *= 1.f / (float)rows;
+        const __nv_bfloat16 b0 = __float2bfloat16_rn(v);
+        const float r1 = v - __bfloat162float(b0);
+        const __nv_bfloat16 b1 = __float2bfloat16_rn(r1);
+        const __nv_bfloat16 b2 = __float2bfloat16_rn(r1 - __bfloat162float(b1));
+        __nv_bfloat16* dst = a.qparts + ((size_t)h * 3 * s.nb + qb) * kD + tid;  // [h][term][nb][128]
+        dst[0] = b0;
+        dst[(size_t)s.nb * kD] = b1;
+        dst[(size_t)2 * s.nb * kD] = b2;
+        const int run_end = min(s.nb, (qb / kProxyChunk + 1) * kProxyChunk);
+        if (tid == 0 && qb == run_end - 1) atomicAdd(a.pooled_cnt + h, 1u);
+      }
+    }
+  }
 }
 
 // RAGGED: n is not a multiple of 128 (separate instance, so the common case keeps the lane-aligned
@@ -171,9 +419,11 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const Shape& s = a.s;
   const int ppg = (s.G + 1) / 2;
-  const int n_items = s.h_kv * ppg * s.n_chunks;
-  const int it0 = (int)((long long)blockIdx.x * n_items / gridDim.x);
-  const int it1 = (int)((long long)(blockIdx.x + 1) * n_items / gridDim.x);
+  const int n_proxy = a.proxy_ctas;
+  const bool pooler = (int)blockIdx.x >= n_proxy;
+  const Sched sched(s, n_proxy, (int)gridDim.x > n_proxy);
+  const int cta = blockIdx.x;
+  const int my_items = pooler ? 0 : sched.count(cta);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
@@ -187,9 +437,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int t = 0; t < 2; ++t)
       for (int b = 0; b < 2; ++b) {
         mbar_init(&sm.s_full[t][b], 1);
-        mbar_init(&sm.s_free[t][b], 4);
+        mbar_init(&sm.s_free[t][b], 8);  // the tile's eight softmax warps
       }
     mbar_init(&sm.mma_done, 1);
+    for (int i = 0; i < POOL_STAGES; ++i) {
+      mbar_init(&sm.pool_full[i], 1);
+      mbar_init(&sm.pool_empty[i], 1);
+    }
     sm.abort = 0;
     fence_mbar_init();
   }
@@ -203,17 +457,22 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  if (warp == PRODUCER_WARP) {
+  if (pooler) {
+    pool_q_blocks(sm, q_map, a, cta - n_proxy, (int)gridDim.x - n_proxy, warp, lane);
+  } else if (warp == PRODUCER_WARP) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&q_map);
       tma_prefetch_desc(&k_map);
       int kc = 0, qn = 0, prev_pair = -1;
       bool ok = true;
-      for (int it = it0; ok && it < it1; ++it) {
-        const Item w(s, it);
+      for (int it = 0; ok && it < my_items; ++it) {
+        int ip, ic;
+        sched.at(cta, it, ip, ic);
+        const Item w(s, ip, ic);
         if (w.pair != prev_pair) {
           // the last 128 queries of each head, once the MMAs on the previous pair's tiles are done
+          trace_mark(a.trace, 0, 0, 1, it);
           if (qn > 0 && !mbar_wait(&sm.q_empty, (qn - 1) & 1, abort)) {
             fail(sm, a.status);
             ok = false;
@@ -229,6 +488,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         for (int j = 0; j < w.nblk; ++j, ++kc) {
           const int st = kc % NS;
+          trace_mark(a.trace, 0, 0, 2, kc);
           if (!mbar_wait(&sm.k_empty[st], ((kc / NS) & 1) ^ 1, abort)) {
             fail(sm, a.status);
             ok = false;
@@ -241,6 +501,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       // Never leave with copies in flight: wait (bounded) for the last load of each stage.
+      trace_mark(a.trace, 0, 0, 3, kc);
       if (qn > 0) mbar_wait(&sm.q_full, (qn - 1) & 1, nullptr);
       for (int j = max(0, kc - NS); j < kc; ++j) mbar_wait(&sm.k_full[j % NS], (j / NS) & 1, nullptr);
     }
@@ -252,10 +513,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       int kc = 0, qn = 0, prev_pair = -1;
       int tb[2] = {0, 0};  // blocks issued per tile so far (S buffer and phase)
       bool ok = true;
-      for (int it = it0; ok && it < it1; ++it) {
-        const Item w(s, it);
+      for (int it = 0; ok && it < my_items; ++it) {
+        int ip, ic;
+        sched.at(cta, it, ip, ic);
+        const Item w(s, ip, ic);
         if (w.pair != prev_pair) {
           if (qn > 0) umma_commit(&sm.q_empty);  // the old Q tiles are free once these MMAs finish
+          trace_mark(a.trace, 0, 1, 1, it);
           if (!mbar_wait(&sm.q_full, qn & 1, abort)) {
             fail(sm, a.status);
             ok = false;
@@ -266,12 +530,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         for (int j = 0; ok && j < w.nblk; ++j, ++kc) {
           const int st = kc % NS;
+          trace_mark(a.trace, 0, 1, 2, kc);
           if (!mbar_wait(&sm.k_full[st], (kc / NS) & 1, abort)) {
             fail(sm, a.status);
             ok = false;
             break;
           }
           for (int t = 0; t < w.ntiles; ++t) {
+            trace_mark(a.trace, 0, 1, 3 + t, tb[t]);
             const int b = tb[t] & 1;
             if (!mbar_wait(&sm.s_free[t][b], ((tb[t] >> 1) & 1) ^ 1, abort)) {
               fail(sm, a.status);
@@ -294,15 +560,19 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       // Never release TMEM under a running MMA: wait (bounded) for all issued work.
+      trace_mark(a.trace, 0, 1, 5, kc);
       umma_commit(&sm.mma_done);
       mbar_wait(&sm.mma_done, 0, nullptr);
+      trace_mark(a.trace, 0, 1, 6, kc);
     }
     __syncwarp();
-  } else if (warp < 8) {
+  } else if (warp < SOFTMAX_WARPS) {
     // ------------------------------------------------------------------ softmax rows
-    const int t = warp >> 2;
-    const int grp = warp & 3;
+    const int t = warp >> 3;           // tile (head of the pair)
+    const int half = (warp >> 2) & 1;  // columns 64*half .. 64*half+63
+    const int grp = warp & 3;          // TMEM lane quarter
     const int r = grp * 32 + lane;
+    const int col0 = 64 * half;
     const uint32_t lane_off = (uint32_t)(grp * 32) << 16;
     // With n = 128 (N_b - 1) + t_last, t_last in [1, 128]: row r sits at position n-128+r, a key
     // at column c of block kb has offset o = n-128+r - 128 kb - c, and the slash block of o is
@@ -313,48 +583,62 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int sigma = (t_last + r) & (kB - 1);
     int tb = 0;  // blocks of this tile so far (S buffer and phase)
     bool ok = true;
-    for (int it = it0; ok && it < it1; ++it) {
-      const Item w(s, it);
-      if (t >= w.ntiles) continue;  // a group's odd last head: this tile has no head here
+    for (int it = 0; ok && it < my_items; ++it) {
+      int ip, ic;
+      sched.at(cta, it, ip, ic);
+      const Item w(s, ip, ic);
+      // (a group's odd last head: tile 1 has no head in its pair)
+      if (t < w.ntiles) {
+      const int h = w.h0 + t;
+      float2* part = a.part + ((size_t)h * s.nb * 2 + half) * kB + r;  // block kb at [kb * 2 * kB]
       float m = -INFINITY;
+      float tot = 0.f;
       float rec = 0.f;  // recency-window mass in block N_b-2 (columns >= t_last), ragged n only
       for (int j = 0; j < w.nblk; ++j, ++tb) {
         const int b = tb & 1;
+        const bool tracer = grp == 0 && lane == 0;
+        if (tracer) trace_mark(a.trace, 0, 2 + t + 2 * half, 1, tb);
         if (!warp_wait(&sm.s_full[t][b], (tb >> 1) & 1, abort)) {
           fail(sm, a.status);
           ok = false;
           break;
         }
         tc_fence_after();
-        // Exponentials use the row reference m of the chunk's earlier blocks without this block's
+        // Exponentials use the segment's reference m of its earlier blocks without this block's
         // maximum (fp32 keeps them exact until they overflow); the first block sets m from its
         // maximum, and a block whose sum would leave [0, 2^64] is redone against its maximum with
-        // the earlier partial sums rescaled. S stays in TMEM until the block is done.
-        const uint32_t sbase = tmem + t * 256 + b * 128 + lane_off;
+        // the earlier sums rescaled. S stays in TMEM until the block is done.
+        const uint32_t sbase = tmem + t * 256 + b * 128 + col0 + lane_off;
         const int kb = w.kb0 + j;
         const int lim = s.n - kB + r - kb * kB;  // row r sees columns c <= lim of this block
         const bool edge = RAGGED ? kb >= s.nb - 2 : kb == s.nb - 1;  // blocks lim can cut
         const bool rec_blk = ragged && s.nb >= 3 && kb == s.nb - 2;
-        bool need_max = (m == -INFINITY);
+        // warp-uniform: the max pass reads TMEM with warp-collective loads, and a row whose half
+        // of the chunk's first block lay wholly beyond its causal limit still has no reference
+        // while the other rows of its warp have one
+        bool need_max = __any_sync(0xffffffffu, m == -INFINITY);
         float lo = 0.f, hi = 0.f, rx = 0.f;
         for (int attempt = 0; attempt < 2; ++attempt) {
           if (need_max) {
-            const float xm = block_max_scaled(sbase, lim, edge);
+            const float xm = block_max_scaled(sbase, col0, lim, edge);
             if (xm > m) {
               const float f = fast_exp2(m - xm);  // 0 while m = -inf
-              for (int jj = 0; jj < j; ++jj) {
-                float2 pv = sm.part[t][jj][r];
-                pv.x *= f;
-                pv.y *= f;
-                sm.part[t][jj][r] = pv;
+              if (m != -INFINITY) {
+                for (int jj = 0; jj < j; ++jj) {  // rare: this thread's earlier sums of the chunk
+                  float2 pv = part[(size_t)(w.kb0 + jj) * 2 * kB];
+                  pv.x *= f;
+                  pv.y *= f;
+                  part[(size_t)(w.kb0 + jj) * 2 * kB] = pv;
+                }
               }
+              tot *= f;
               rec *= f;
               m = xm;
             }
           }
           const float nm = -m;
           if (!RAGGED && !edge) {
-            block_sums_fast(sbase, nm, grp, lane, lo, hi);
+            block_sums_fast(sbase, nm, grp, lane, half, lo, hi);
           } else {
             // hardware exp2 only, every column tested against the causal limit and (n not a
             // multiple of 128) the split column, which is not aligned with the lanes
@@ -362,13 +646,13 @@ __global__ void __launch_bounds__(THREADS, 1)
             hi = 0.f;
             rx = 0.f;
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
               uint32_t v[32];
               tmem_ld32(sbase + c * 32, v);
               tmem_ld_wait_regs(v);
 #pragma unroll
               for (int q = 0; q < 32; ++q) {
-                const int col = c * 32 + q;
+                const int col = col0 + c * 32 + q;
                 float e = fast_exp2(fmaf(__uint_as_float(v[q]), kScaleLog2, nm));
                 if (edge && col > lim) e = 0.f;  // causal: row r sees keys up to its own position
                 const bool low = RAGGED ? col <= sigma : col <= r;
@@ -384,22 +668,21 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.s_free[t][b]);
-        sm.part[t][j][r] = make_float2(lo, hi);
+        part[(size_t)kb * 2 * kB] = make_float2(lo, hi);
+        tot += lo + hi;
         if (rec_blk) rec = rx;
       }
-      if (!ok) break;
-      const int h = w.h0 + t;
-      float tot = 0.f;
-      for (int jj = 0; jj < w.nblk; ++jj) {
-        const float2 pv = sm.part[t][jj][r];
-        a.part[((size_t)h * s.nb + w.kb0 + jj) * kB + r] = pv;
-        tot += pv.x + pv.y;
+      if (ok) {
+        // the segment (chunk, half): its reference and total per row
+        const size_t ci = (((size_t)h * s.n_chunks + w.chunk) * 2 + half) * kB + r;
+        a.chunk_max[ci] = m;
+        a.chunk_tot[ci] = tot;
+        if (ragged && s.nb >= 3 && s.nb - 2 >= w.kb0 && s.nb - 2 < w.kb0 + w.nblk)
+          a.rec_extra[((size_t)h * 2 + half) * kB + r] = rec;
       }
-      const size_t ci = ((size_t)h * s.n_chunks + w.chunk) * kB + r;
-      a.chunk_max[ci] = m;
-      a.chunk_tot[ci] = tot;
-      if (ragged && s.nb >= 3 && s.nb - 2 >= w.kb0 && s.nb - 2 < w.kb0 + w.nblk)
-        a.rec_extra[(size_t)h * kB + r] = rec;
+      }
+      // every softmax warp takes part, whether or not its tile had a head or an error occurred
+      if (sched.is_anchor(cta, it)) anchor_done(sm, a, w, sched.apc, t, half, grp, lane);
     }
     __syncwarp();
   } else if (warp >= POOL_WARP) {
@@ -411,8 +694,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int pw = warp - POOL_WARP;
     int kc = 0;
     bool ok = true;
-    for (int it = it0; ok && it < it1; ++it) {
-      const Item w(s, it);
+    for (int it = 0; ok && it < my_items; ++it) {
+      int ip, ic;
+      sched.at(cta, it, ip, ic);
+      const Item w(s, ip, ic);
       const int ncc_item = (16 - w.pig + ppg - 1) / ppg;
       const int ncc = (ncc_item - pw + 1) / 2;
       int groups = 1;
@@ -424,6 +709,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int half = cc >> 3, ch = cc & 7;
       for (int j = 0; j < w.nblk; ++j, ++kc) {
         const int st = kc % NS;
+        if (lane == 0 && pw == 0) trace_mark(a.trace, 0, 6, 1, kc);
         if (!warp_wait(&sm.k_full[st], (kc / NS) & 1, abort)) {
           fail(sm, a.status);
           ok = false;
@@ -493,6 +779,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncwarp();
   }
 
+  if (lane == 0 && (warp == PRODUCER_WARP || warp == MMA_WARP || warp == 0 || warp == 8 || warp == POOL_WARP))
+    trace_mark(a.trace, 0, 7, 7, warp);
   tc_fence_before();
   __syncthreads();
   if (warp == MMA_WARP) {
@@ -521,9 +809,22 @@ cudaError_t launch_proxy_pass(const CUtensorMap& q_map, const CUtensorMap& k_map
   auto kernel = ragged ? proxy_pass_kernel<true> : proxy_pass_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int n_items = a.s.h_kv * ((a.s.G + 1) / 2) * a.s.n_chunks;
-  dim3 grid(min(n_items, num_sms()));  // persistent: one CTA per SM, a run of items each
-  kernel<<<grid, THREADS, smem, st>>>(q_map, k_map, a);
+  // Persistent: one CTA per SM. With the C_struct router a share of the SMs pools Q_bar of the
+  // heads the anchor chunks already show to be Pooled-Estimation, while the rest run the proxy
+  // items; the anchor items go first so the hints come early.
+  const int pairs = a.s.h_kv * ((a.s.G + 1) / 2);
+  const int n_items = pairs * a.s.n_chunks;
+  const int n_anchor = pairs * min(2, a.s.n_chunks);
+  const int sms = num_sms();
+  int n_pool = a.route_rule == 0 ? (sms * kPoolShareNum) / kPoolShareDen : 0;
+  int n_proxy = min(n_items, sms - n_pool);
+  if (n_anchor > n_proxy || n_pool <= 0) {
+    n_pool = 0;
+    n_proxy = min(n_items, sms);
+  }
+  SelectArgs args = a;
+  args.proxy_ctas = n_proxy;
+  kernel<<<n_proxy + n_pool, THREADS, smem, st>>>(q_map, k_map, args);
   return cudaGetLastError();
 }
 

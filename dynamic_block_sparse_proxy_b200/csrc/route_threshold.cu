@@ -1,8 +1,8 @@
 // route_threshold.cu — per-head routing and the Vertical-Slash noise-floor rule.
 //
 // Inputs are the proxy pass's per-(row, key block) split sums, each relative to its chunk's
-// reference row maximum. One kernel: row statistics and block masses over many CTAs per head,
-// and the head's last CTA takes the decisions:
+// reference row maximum. Row statistics (one CTA per head), then block masses over many CTAs per
+// head, the head's last CTA taking the decisions:
 //   1. per proxy row r: global max M_r and normaliser Z_r over all chunks, and the weight
 //      w = exp2(m_chunk - M_r) / (Z_r * B) that turns a chunk's sums into column-mean mass;
 //   2. p_v[kb] = sum_r w*(lo+hi) (vertical block mass), and the slash block masses
@@ -255,9 +255,13 @@ __device__ void route_head(const SelectArgs& a, int h) {
   double C = nb >= 2 ? pv[0] + pv[nb - 1] : pv[0];
   const int t_last = s.n - (nb - 1) * kB;
   if (t_last != kB && nb >= 3) {
-    const float* wr = a.row_w + ((size_t)h * s.n_chunks + (nb - 2) / kProxyChunk) * kB;
+    // both 64-column halves of block N_b-2, each with its segment's weight
     double x = 0.0;
-    for (int r = tid; r < kB; r += THREADS) x += (double)a.rec_extra[(size_t)h * kB + r] * (double)__ldcg(wr + r);
+    for (int i = tid; i < 2 * kB; i += THREADS) {
+      const int half = i / kB, r = i % kB;
+      const float* wr = a.row_w + (((size_t)h * s.n_chunks + (nb - 2) / kProxyChunk) * 2 + half) * kB;
+      x += (double)a.rec_extra[((size_t)h * 2 + half) * kB + r] * (double)__ldcg(wr + r);
+    }
     C += block_sum(x, red);
   }
   double jsd = 0.0;
@@ -352,16 +356,80 @@ __device__ void route_head(const SelectArgs& a, int h) {
 }
 
 // 1-2. One CTA per run of MASS_BLOCKS key blocks of a head:
-//   (a) per proxy row r: the global reference max M_r over the chunks, the normaliser Z_r, and
-//       for the CTA's chunks the weight w = exp2(m_chunk - M_r) / (Z_r * B) that turns a chunk's
-//       sums into column-mean mass (four threads per row, fp64 sums);
-//   (b) block masses, one warp per key block: p_v[kb] = sum_r w*(lo+hi). A row r whose split
+//   (a) per proxy row r: the global reference max M_r over the segments (the proxy pass keeps
+//       one reference per chunk and 64-column half), the normaliser Z_r, and for the CTA's
+//       segments the weight w = exp2(m_seg - M_r) / (Z_r * B) that turns a segment's sums into
+//       column-mean mass (four threads per row, fp64 sums);
+//   (b) block masses, one warp per key block: p_v[kb] = sum_r sum_half w*(lo+hi). A row r whose split
 //       column is (t_last + r) mod 128 (t_last = n - 128 (N_b-1), 128 when n is a multiple of
 //       128) meets slash blocks N_b-1-kb (lo) and N_b-2-kb (hi) when t_last + r >= 128, else
 //       N_b-2-kb (lo) and N_b-3-kb (hi) (CRISP §4, both directions). Every slot of ps_lo, ps_hi
 //       and ps_x is written once: by the key block that maps there, or with 0 by the block whose
 //       target lies below 0;
 //   (c) the head's last CTA to finish routes the head (route_head).
+// 1. Per proxy row r: the global reference max M_r over the segments (the proxy pass keeps one
+//    reference per chunk and 64-column half), the normaliser Z_r (fp64), and for every segment
+//    the weight w = exp2(m_seg - M_r) / (Z_r * B) that turns the segment's sums into column-mean
+//    mass. One CTA per (32 rows, head); thread (part, row) takes segments part, part+16, ..., all
+//    of its loads in flight before the first use.
+constexpr int STAT_ROWS = 32;
+constexpr int STAT_PARTS = THREADS / STAT_ROWS;  // 16
+constexpr int STAT_UNROLL = 8;
+__global__ void __launch_bounds__(THREADS) row_stats_kernel(const SelectArgs a) {
+  const Shape& s = a.s;
+  const int h = blockIdx.y, tid = threadIdx.x;
+  const int r = blockIdx.x * STAT_ROWS + (tid % STAT_ROWS), part = tid / STAT_ROWS;
+  const int nseg = 2 * s.n_chunks;
+  const float* mc = a.chunk_max + (size_t)h * nseg * kB + r;
+  const float* tc = a.chunk_tot + (size_t)h * nseg * kB + r;
+  __shared__ float smax[STAT_PARTS][STAT_ROWS];
+  __shared__ double ssum[STAT_PARTS][STAT_ROWS];
+  float M = -INFINITY;
+  for (int g0 = part; g0 < nseg; g0 += STAT_PARTS * STAT_UNROLL) {
+    float x[STAT_UNROLL];
+#pragma unroll
+    for (int u = 0; u < STAT_UNROLL; ++u) {
+      const int g = g0 + STAT_PARTS * u;
+      x[u] = g < nseg ? mc[(size_t)g * kB] : -INFINITY;
+    }
+#pragma unroll
+    for (int u = 0; u < STAT_UNROLL; ++u) M = fmaxf(M, x[u]);
+  }
+  smax[part][tid % STAT_ROWS] = M;
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < STAT_PARTS; ++i) M = fmaxf(M, smax[i][tid % STAT_ROWS]);
+  double Z = 0.0;
+  for (int g0 = part; g0 < nseg; g0 += STAT_PARTS * STAT_UNROLL) {
+    float x[STAT_UNROLL], y[STAT_UNROLL];
+#pragma unroll
+    for (int u = 0; u < STAT_UNROLL; ++u) {
+      const int g = g0 + STAT_PARTS * u;
+      x[u] = g < nseg ? mc[(size_t)g * kB] : -INFINITY;
+      y[u] = g < nseg ? tc[(size_t)g * kB] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < STAT_UNROLL; ++u)
+      if (g0 + STAT_PARTS * u < nseg) Z += (double)exp2f(x[u] - M) * (double)y[u];
+  }
+  ssum[part][tid % STAT_ROWS] = Z;
+  __syncthreads();
+  Z = 0.0;
+#pragma unroll
+  for (int i = 0; i < STAT_PARTS; ++i) Z += ssum[i][tid % STAT_ROWS];
+  const double inv = 1.0 / (Z * kB);
+  float* wr = a.row_w + (size_t)h * nseg * kB + r;
+  for (int g = part; g < nseg; g += STAT_PARTS) wr[(size_t)g * kB] = (float)((double)exp2f(mc[(size_t)g * kB] - M) * inv);
+}
+
+// 2-3. One CTA per run of MASS_BLOCKS key blocks of a head:
+//   (a) block masses, one warp per key block: p_v[kb] = sum_r sum_half w*(lo+hi). A row r whose
+//       split column is (t_last + r) mod 128 (t_last = n - 128 (N_b-1), 128 when n is a multiple
+//       of 128) meets slash blocks N_b-1-kb (lo) and N_b-2-kb (hi) when t_last + r >= 128, else
+//       N_b-2-kb (lo) and N_b-3-kb (hi) (CRISP §4, both directions). Every slot of ps_lo, ps_hi
+//       and ps_x is written once: by the key block that maps there, or with 0 by the block whose
+//       target lies below 0;
+//   (b) the head's last CTA to finish routes the head (route_head).
 constexpr int MASS_BLOCKS = 64;                     // key blocks per CTA
 constexpr int MASS_CHUNKS = MASS_BLOCKS / kProxyChunk;
 __global__ void __launch_bounds__(THREADS) mass_route_kernel(const SelectArgs a) {
@@ -369,40 +437,34 @@ __global__ void __launch_bounds__(THREADS) mass_route_kernel(const SelectArgs a)
   const int h = blockIdx.y, nb = s.nb, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int kb0 = blockIdx.x * MASS_BLOCKS;
   const int c0 = kb0 / kProxyChunk, c1 = min(s.n_chunks, c0 + MASS_CHUNKS);
-  __shared__ float w_s[MASS_CHUNKS][kB];
-  {
-    const int r = tid >> 2, part = tid & 3;  // four threads per row, chunks part, part+4, ...
-    const float* mc = a.chunk_max + (size_t)h * s.n_chunks * kB;
-    const float* tc = a.chunk_tot + (size_t)h * s.n_chunks * kB;
-    float M = -INFINITY;
-    for (int c = part; c < s.n_chunks; c += 4) M = fmaxf(M, mc[c * kB + r]);
-    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 1));
-    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 2));
-    double Z = 0.0;
-    for (int c = part; c < s.n_chunks; c += 4) Z += (double)exp2f(mc[c * kB + r] - M) * (double)tc[c * kB + r];
-    Z += __shfl_xor_sync(0xffffffffu, Z, 1);
-    Z += __shfl_xor_sync(0xffffffffu, Z, 2);
-    const double inv = 1.0 / (Z * kB);
-    const int c = c0 + part;
-    if (c < c1) {
-      const float w = (float)((double)exp2f(mc[c * kB + r] - M) * inv);
-      w_s[part][r] = w;
-      a.row_w[((size_t)h * s.n_chunks + c) * kB + r] = w;
-    }
-  }
+  const int nseg = 2 * s.n_chunks;
+  __shared__ float w_s[2 * MASS_CHUNKS][kB];
+  for (int i = tid; i < 2 * (c1 - c0) * kB; i += THREADS)
+    w_s[i / kB][i % kB] = a.row_w[((size_t)h * nseg + 2 * c0) * kB + i];
   __syncthreads();
   const int t_last = s.n - (nb - 1) * kB;
-  for (int kb = kb0 + warp; kb < min(nb, kb0 + MASS_BLOCKS); kb += NWARP) {
-    const float2* p = a.part + ((size_t)h * nb + kb) * kB;
-    const float* wc = w_s[kb / kProxyChunk - c0];
+  // each warp's key blocks kb0 + warp + 16 i, two at a time with both blocks' sums loaded
+  // before the first is used
+  for (int k0 = 0; k0 < MASS_BLOCKS / NWARP; k0 += 2) {
+  float2 vv[2][2 * kB / 32];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int kb = kb0 + warp + NWARP * (k0 + k);
+#pragma unroll
+    for (int i = 0; i < 2 * kB / 32; ++i)
+      vv[k][i] = kb < nb ? a.part[(size_t)(h * nb + kb) * 2 * kB + lane + 32 * i] : make_float2(0.f, 0.f);
+  }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int kb = kb0 + warp + NWARP * (k0 + k);
+    if (kb >= nb) break;
+    const float* wc = w_s[2 * (kb / kProxyChunk - c0)];         // [half][128]
     double loA = 0.0, hiA = 0.0, loB = 0.0, hiB = 0.0;
-    float2 v[kB / 32];
+    const float2* v = vv[k];
 #pragma unroll
-    for (int i = 0; i < kB / 32; ++i) v[i] = p[lane + 32 * i];
-#pragma unroll
-    for (int i = 0; i < kB / 32; ++i) {
-      const int r = lane + 32 * i;
-      const double ww = wc[r];
+    for (int i = 0; i < 2 * kB / 32; ++i) {
+      const int r = (lane + 32 * i) & (kB - 1);
+      const double ww = wc[lane + 32 * i];
       if (t_last + r >= kB) {
         loA += (double)v[i].x * ww;
         hiA += (double)v[i].y * ww;
@@ -428,6 +490,7 @@ __global__ void __launch_bounds__(THREADS) mass_route_kernel(const SelectArgs a)
       else a.ps_x[base + (nb - 3 - kb == -1 ? nb - 2 : nb - 1)] = 0.0;  // kb = N_b-2, N_b-1
     }
   }
+  }
   // the head's last CTA routes it (counter back to zero for the radix levels that reuse it)
   __threadfence();
   __syncthreads();
@@ -446,6 +509,7 @@ cudaError_t launch_route_threshold(const SelectArgs& a, cudaStream_t st) {
   const size_t smem = (size_t)3 * a.s.nb * sizeof(double);  // p_v, p_s, and a_bar / sort indices
   cudaError_t e = cudaFuncSetAttribute(mass_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  row_stats_kernel<<<dim3(kB / STAT_ROWS, a.s.h_q), THREADS, 0, st>>>(a);
   mass_route_kernel<<<dim3((a.s.nb + MASS_BLOCKS - 1) / MASS_BLOCKS, a.s.h_q), THREADS, smem, st>>>(a);
   return cudaGetLastError();
 }
