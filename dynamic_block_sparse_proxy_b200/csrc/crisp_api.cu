@@ -130,10 +130,6 @@ int run_select(const void* q, const void* k, const Shape& s, const crisp_params*
   a.hist_mass = at<unsigned long long>(ws, w.hist_mass);
   a.cut = at<CutState>(ws, w.cut);
   a.cut_done = at<uint32_t>(ws, w.cut_done);
-  a.anchor_cnt = at<uint32_t>(ws, w.anchor_cnt);
-  a.hint = at<uint32_t>(ws, w.hint);
-  a.hint_ready = at<uint32_t>(ws, w.hint_ready);
-  a.pooled_cnt = at<uint32_t>(ws, w.pooled_cnt);
   a.keep_v = at<uint8_t>(ws, w.keep_v);
   a.keep_s = at<uint8_t>(ws, w.keep_s);
   a.cnt = at<int>(ws, w.cnt);
@@ -155,10 +151,9 @@ int run_select(const void* q, const void* k, const Shape& s, const crisp_params*
   if (rc == CRISP_OK) rc = make_map3(&kpm, a.kparts, (uint64_t)s.nb, (uint64_t)s.h_kv * 3, (uint64_t)s.nb);
   if (rc != CRISP_OK) return rc;
 
-  // The radix histograms accumulate with atomics, the cut levels count finished CTAs, and the
-  // proxy pass's early pooling keeps counters and flags: start from zero (the arrays are
-  // contiguous).
-  if (cudaMemsetAsync(at<uint8_t>(ws, w.hist_cnt), 0, w.pooled_cnt + (size_t)s.h_q * 4 - w.hist_cnt, st) != cudaSuccess)
+  // The radix histograms accumulate with atomics and the cut levels count finished CTAs: start
+  // from zero (the arrays are contiguous).
+  if (cudaMemsetAsync(at<uint8_t>(ws, w.hist_cnt), 0, w.cut_done + (size_t)s.h_q * 4 - w.hist_cnt, st) != cudaSuccess)
     return CRISP_ERR_CUDA;
   if (launch_proxy_pass(qm, km, a, st) != cudaSuccess) return CRISP_ERR_CUDA;
   if (launch_route_threshold(a, st) != cudaSuccess) return CRISP_ERR_CUDA;

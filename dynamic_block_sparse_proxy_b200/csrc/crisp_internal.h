@@ -39,7 +39,7 @@ struct CutState {
 
 struct Workspace {
   size_t status, trace, part, chunk_max, chunk_tot, row_w, pv, ps_lo, ps_hi, ps_x, rec_extra, kbar, kparts, qparts,
-      pbuf, hist_cnt, hist_mass, cut, cut_done, anchor_cnt, hint, hint_ready, pooled_cnt, keep_v, keep_s, cnt,
+      pbuf, hist_cnt, hist_mass, cut, cut_done, keep_v, keep_s, cnt,
       eqcnt, eqbase, selmask, idx_route, idx_c, idx_row_ptr, idx_cols, total;
 };
 
@@ -73,15 +73,11 @@ inline Workspace workspace_layout(const Shape& s) {
   w.kparts = take((size_t)s.h_kv * 3 * nb * kD * 2);
   w.qparts = take(hq * 3 * nb * kD * 2);
   w.pbuf = take(hq * (size_t)s.cap * 4);
-  // hist_cnt .. pooled_cnt are contiguous: one memset clears them at the start of a selection
+  // hist_cnt .. cut_done are contiguous: one memset clears them at the start of a selection
   w.hist_cnt = take(hq * kHistBins * 4);
   w.hist_mass = take(hq * kHistBins * 8);
   w.cut = take(hq * sizeof(CutState));
   w.cut_done = take(hq * 4);
-  w.anchor_cnt = take(hq * 4);
-  w.hint = take(hq * 4);
-  w.hint_ready = take(hq * 4);
-  w.pooled_cnt = take(hq * 4);
   w.keep_v = take(hq * nb);
   w.keep_s = take(hq * nb);
   w.cnt = take(hq * nb * 4);
@@ -124,13 +120,6 @@ struct SelectArgs {
   unsigned long long* hist_mass;  // fixed point, 2^-40 units
   CutState* cut;
   uint32_t* cut_done;           // per head: CTAs of the current radix level that finished
-  // Q_bar pooling during the proxy pass (see proxy_pass.cu): per head pair, anchor chunks done;
-  // per head, the early Pooled-Estimation hint, its ready flag, and the 16-block runs pooled
-  uint32_t* anchor_cnt;
-  uint32_t* hint;
-  uint32_t* hint_ready;
-  uint32_t* pooled_cnt;
-  int proxy_ctas;               // CTAs of the proxy pass that run proxy items (the rest pool Q_bar)
   uint8_t* keep_v;
   uint8_t* keep_s;
   int* cnt;
@@ -167,6 +156,9 @@ cudaError_t launch_merge(const SelectArgs& a, cudaStream_t st);
 cudaError_t launch_sparse_attn(const CUtensorMap& q_map, const CUtensorMap& k_map,
                                const CUtensorMap& v_map, const AttnArgs& a, cudaStream_t st);
 cudaError_t launch_timeout_selftest(int* status, unsigned long long limit_ns, cudaStream_t st);
+
+// SMs of the current device (queried once).
+int num_sms();
 
 // Host-side helpers shared by the entry points (crisp_api.cu).
 int check_shape(int h_q, int h_kv, int n, int d, Shape* s);

@@ -5,8 +5,7 @@
 // For every head routed to PE:
 //   qbar_kernel     Q_bar[qb] = mean of the block's query rows (fp32; 128, or fewer in a partial
 //                   last block), read once from HBM, stored as three bf16 terms whose sum is the
-//                   fp32 value exactly (hi, mid, lo) — for the PE heads the proxy pass did not
-//                   already pool while it ran;
+//                   fp32 value exactly (hi, mid, lo);
 //   scores_kernel   logits Q_bar[qb] . K_bar[kb] / sqrt(d) for kb <= qb, one 128x128 tile per
 //                   CTA on the tensor cores: the six products hi.hi + hi.mid + mid.hi + hi.lo +
 //                   mid.mid + lo.hi of the split operands accumulate in fp32 in TMEM (the terms
@@ -44,8 +43,6 @@ __global__ void __launch_bounds__(128) qbar_kernel(const SelectArgs a) {
   const int qb = blockIdx.x, h = blockIdx.y;
   if (!is_pe(a, h)) return;
   const Shape& s = a.s;
-  // heads the proxy pass pooled already (every run of 16 query blocks counted)
-  if (a.pooled_cnt[h] == (uint32_t)((s.nb + kProxyChunk - 1) / kProxyChunk)) return;
   const int t = threadIdx.x, c16 = t & 15, rg = t >> 4;
   const __nv_bfloat16* base = a.q + ((size_t)h * s.ld + (size_t)qb * kB) * kD + c16 * 8;
   float acc[8];
@@ -231,33 +228,29 @@ __device__ __forceinline__ unsigned long long to_fixed(float p) {
   return q + ((rem > half || (rem == half && (q & 1ull))) ? 1ull : 0ull);
 }
 
-// Per-lane run of histogram updates: consecutive entries of one lane that fall in the same bin are
-// counted and summed in registers and go to shared memory (two atomics) only when the bin
-// changes. A pooled row's probabilities mostly share a few bins, so a lane flushes a few times
-// per row.
-struct BinRun {
-  uint32_t bin = 0xffffffffu, cnt = 0u;
-  unsigned long long mass = 0ull;
-  __device__ __forceinline__ void add(uint32_t* scnt, unsigned long long* smass, uint32_t b, unsigned long long fx) {
-    if (b != bin) {
-      flush(scnt, smass);
-      bin = b;
-    }
-    ++cnt;
-    mass += fx;
+// Level-1 histogram of one row step (all lanes call it): only the mass of a bin decides the
+// level-1 choice (the chosen bin's mass is positive, so it holds entries), so level 1 keeps no
+// counts. Lanes with the same bin form a group (match.any); each group sums its fixed-point masses
+// as three 16-bit parts (redux.sync, one instruction per part for every group at once) and its
+// lowest lane adds them to three 32-bit shared arrays: no 64-bit shared atomics, and no two lanes
+// of a warp hit the same word. A CTA's part sums stay below 2^32 (at most 8192 entries of < 2^16).
+__device__ __forceinline__ void warp_mass_add(uint32_t (*smass3)[kHistBins], bool valid, float p) {
+  const unsigned long long fx = valid ? to_fixed(p) : 0ull;
+  const uint32_t key = fx != 0ull ? (__float_as_uint(p) >> 20) : 0xffffffffu;
+  const unsigned grp = __match_any_sync(0xffffffffu, key);
+  const uint32_t s0 = __reduce_add_sync(grp, (uint32_t)(fx & 0xffffu));
+  const uint32_t s1 = __reduce_add_sync(grp, (uint32_t)((fx >> 16) & 0xffffu));
+  const uint32_t s2 = __reduce_add_sync(grp, (uint32_t)(fx >> 32));
+  if (key != 0xffffffffu && (threadIdx.x & 31) == __ffs(grp) - 1) {
+    atomicAdd(&smass3[0][key], s0);
+    atomicAdd(&smass3[1][key], s1);
+    atomicAdd(&smass3[2][key], s2);
   }
-  __device__ __forceinline__ void flush(uint32_t* scnt, unsigned long long* smass) {
-    if (cnt) {
-      atomicAdd(&scnt[bin], cnt);
-      atomicAdd(&smass[bin], mass);
-    }
-    cnt = 0u;
-    mass = 0ull;
-  }
-};
+}
 
-// Adds a CTA's shared histogram to the head's global one, then reports whether this CTA is the
-// last of the head's `ctas` to finish (that CTA then sees every CTA's counts).
+// Adds a CTA's shared histogram (nbins bins of counts and masses) to the head's global one, then
+// reports whether this CTA is the last of the head's `ctas` to finish (that CTA then sees every
+// CTA's updates).
 __device__ bool flush_and_check_last(const SelectArgs& a, int h, const uint32_t* scnt,
                                      const unsigned long long* smass, int nbins, int ctas) {
   uint32_t* gcnt = a.hist_cnt + (size_t)h * kHistBins;
@@ -344,7 +337,8 @@ __device__ void select_bin(const SelectArgs& a, int h, int level) {
       if (k < per) {
         const unsigned long long hi = suf;
         suf += mb[k];
-        if (above + suf >= target && above + hi < target && cb[k] > 0) atomicMax(&found, b0 + k);
+        // (both hold only if the bin's mass is positive: it holds entries)
+        if (above + suf >= target && above + hi < target) atomicMax(&found, b0 + k);
       }
     }
     __syncthreads();
@@ -391,7 +385,7 @@ __device__ void select_bin(const SelectArgs& a, int h, int level) {
 }
 
 // One warp per pooled row (8 rows per CTA): P[qb, kb] = softmax over kb <= qb, in place, and
-// the level-1 histogram (bits 30..20 of the positive fp32 pattern). A row of up to 1024 entries
+// the level-1 mass histogram (bits 30..20 of the positive fp32 pattern). A row of up to 1024 entries
 // stays in registers (32 per lane, all loads in flight at once); longer rows take three passes
 // over memory. Exponentials use the exp2 unit on log2(e)-scaled logits.
 constexpr int ROWS_PER_CTA = 8;
@@ -399,12 +393,8 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32, 4) rowsoft_kernel(const Sel
   const int h = blockIdx.y;
   if (!is_pe(a, h)) return;
   const Shape& s = a.s;
-  __shared__ uint32_t scnt[kHistBins];
-  __shared__ unsigned long long smass[kHistBins];
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) {
-    scnt[i] = 0;
-    smass[i] = 0ull;
-  }
+  __shared__ uint32_t smass3[3][kHistBins];  // 16-bit parts of the fixed-point bin masses
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) smass3[0][i] = smass3[1][i] = smass3[2][i] = 0u;
   __syncthreads();
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int qb = blockIdx.x * ROWS_PER_CTA + w;
@@ -436,17 +426,15 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32, 4) rowsoft_kernel(const Sel
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
       const float inv = 1.f / z;
-      BinRun run;
 #pragma unroll
       for (int u = 0; u < 32; ++u) {
-        const int i = u * 32 + lane;
-        if (u * 32 < L && i < L) {
+        if (u * 32 < L) {
+          const int i = u * 32 + lane;
           const float p = x[u] * inv;
-          row[i] = p;
-          run.add(scnt, smass, __float_as_uint(p) >> 20, to_fixed(p));
+          if (i < L) row[i] = p;
+          warp_mass_add(smass3, i < L, p);
         }
       }
-      run.flush(scnt, smass);
     } else {
       float mx = -INFINITY;
       for (int base = 0; base < L; base += 256) {
@@ -482,7 +470,6 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32, 4) rowsoft_kernel(const Sel
       for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
       const float inv = 1.f / z;
       __syncwarp();
-      BinRun run;
       for (int base = 0; base < L; base += 256) {
         float e[8];
 #pragma unroll
@@ -493,18 +480,21 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32, 4) rowsoft_kernel(const Sel
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const int i = base + 32 * u + lane;
-          if (i < L) {
-            const float p = e[u] * inv;
-            row[i] = p;
-            run.add(scnt, smass, __float_as_uint(p) >> 20, to_fixed(p));
-          }
+          const float p = e[u] * inv;
+          if (i < L) row[i] = p;
+          warp_mass_add(smass3, i < L, p);
         }
       }
-      run.flush(scnt, smass);
     }
   }
   __syncthreads();
-  if (flush_and_check_last(a, h, scnt, smass, kHistBins, gridDim.x)) select_bin(a, h, 1);
+  // the CTA's bin masses (the parts recombined), then its share of the global histogram
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) {
+    const unsigned long long m = (unsigned long long)smass3[0][i] + ((unsigned long long)smass3[1][i] << 16) +
+                                 ((unsigned long long)smass3[2][i] << 32);
+    if (m) atomicAdd(a.hist_mass + (size_t)h * kHistBins + i, m);
+  }
+  if (flush_and_check_last(a, h, nullptr, nullptr, 0, gridDim.x)) select_bin(a, h, 1);
 }
 
 // --------------------------------------------------------------------- histogram, levels 2-3

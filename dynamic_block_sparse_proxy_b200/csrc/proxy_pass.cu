@@ -45,23 +45,9 @@ constexpr uint32_t TILE_BYTES = kB * kD * 2;
 constexpr uint32_t HALF_BYTES = TILE_BYTES / 2;
 constexpr float kScaleLog2 = 0.12751743074380045f;  // log2(e) / sqrt(128)
 
-constexpr int POOL_STAGES = 5;  // Q blocks in flight in a pooling CTA (over the q and k buffers)
-// Share of the SMs that pool Q_bar during the proxy pass (numerator / denominator).
-#ifndef CRISP_POOL_SHARE_NUM
-#define CRISP_POOL_SHARE_NUM 16
-#endif
-constexpr int kPoolShareNum = CRISP_POOL_SHARE_NUM;
-constexpr int kPoolShareDen = 100;
-
 struct __align__(1024) ProxySmem {
   __nv_bfloat16 q[2][kB * kD];  // two 128-byte-swizzled halves [128 rows][64 cols] per tile
   __nv_bfloat16 k[NS][kB * kD];
-  float red[2][32][kD];         // pooling CTAs: per-row-group partial sums of a Q block
-  uint64_t pool_full[POOL_STAGES];
-  uint64_t pool_empty[POOL_STAGES];
-  int stage_info[POOL_STAGES];  // head * 65536 + query block of the stage, or -1: no more
-  float hint_part[2][4];
-  int anchor_last;
   uint64_t q_full;
   uint64_t q_empty;
   uint64_t k_full[NS];
@@ -108,42 +94,22 @@ struct Item {
   }
 };
 
-// Which items a proxy CTA runs. The items are the (head pair, chunk) pairs; CTA c runs a
-// contiguous share of them. With early pooling ("anchored"), CTA c < A first runs anchor item c
-// — the chunks holding a pair's sink block (chunk 0) and last block (chunk n_chunks-1), which
-// bound the pair's C_struct from above — and then its share of the other items, listed pair by
-// pair; otherwise its share of the pair-major list.
+// Which items a CTA runs: the items are the (head pair, chunk) pairs listed pair by pair; CTA c
+// of P runs the contiguous share [c I / P, (c+1) I / P).
 struct Sched {
-  int I, A, apc, nac, n_proxy, n_chunks;
-  bool anchored;
-  __device__ __forceinline__ Sched(const Shape& s, int n_proxy_, bool anchored_) {
-    const int pairs = s.h_kv * ((s.G + 1) / 2);
+  int I, P, n_chunks;
+  __device__ __forceinline__ Sched(const Shape& s, int P_) {
     n_chunks = s.n_chunks;
-    I = pairs * n_chunks;
-    apc = min(2, n_chunks);
-    A = pairs * apc;
-    nac = n_chunks - apc;
-    n_proxy = n_proxy_;
-    anchored = anchored_;
+    I = s.h_kv * ((s.G + 1) / 2) * n_chunks;
+    P = P_;
   }
   __device__ __forceinline__ int count(int c) const {
-    return (int)(((long long)(c + 1) * I) / n_proxy - ((long long)c * I) / n_proxy);
+    return (int)(((long long)(c + 1) * I) / P - ((long long)c * I) / P);
   }
-  __device__ __forceinline__ bool is_anchor(int c, int k) const { return anchored && c < A && k == 0; }
   __device__ __forceinline__ void at(int c, int k, int& pair, int& chunk) const {
-    const long long start = ((long long)c * I) / n_proxy;
-    if (!anchored) {
-      const long long it = start + k;
-      pair = (int)(it / n_chunks);
-      chunk = (int)(it % n_chunks);
-    } else if (c < A && k == 0) {
-      pair = c / apc;
-      chunk = (c % apc == 0) ? n_chunks - 1 : 0;
-    } else {
-      const long long x = start - min(c, A) + k - (c < A ? 1 : 0);  // index among the other items
-      pair = (int)(x / nac);
-      chunk = 1 + (int)(x % nac);
-    }
+    const long long it = ((long long)c * I) / P + k;
+    pair = (int)(it / n_chunks);
+    chunk = (int)(it % n_chunks);
   }
 };
 
@@ -219,193 +185,6 @@ __device__ __forceinline__ float block_max_scaled(uint32_t sbase, int col0, int 
   return mx * kScaleLog2;
 }
 
-// End of an anchor item (run by all 16 softmax warps): the CTA that completes the second anchor
-// chunk of a head pair computes, for each of the pair's heads, an upper bound of its C_struct from
-// the two anchor chunks alone — the mass of the first and last 128 keys over the mass of the
-// anchor chunks' keys, whose total can only grow with the other chunks — and publishes
-// hint[h] = 1 (Pooled-Estimation for sure, up to rounding) when the bound is below tau_proxy.
-// Pooling CTAs start on Q_bar of hinted heads while the other chunks run. The hint only decides
-// when Q_bar is pooled, never a route.
-__device__ void anchor_done(ProxySmem& sm, const SelectArgs& a, const Item& w, int apc, int t, int half, int grp,
-                            int lane) {
-  const Shape& s = a.s;
-  __threadfence();  // this thread's sums and segment statistics, before the count
-  named_bar_sync(1, SOFTMAX_WARPS * 32);
-  if (threadIdx.x == 0) {
-    const bool aborted = *reinterpret_cast<volatile int*>(&sm.abort) != 0;
-    sm.anchor_last = (!aborted && atomicAdd(a.anchor_cnt + w.pair, 1u) == (unsigned)(apc - 1)) ? 1 : 0;
-  }
-  named_bar_sync(1, SOFTMAX_WARPS * 32);
-  if (!sm.anchor_last) return;
-  __threadfence();  // the other anchor's writes are visible
-  const int nb = s.nb, nch = s.n_chunks, last = nch - 1;
-  if (half == 0 && t < w.ntiles) {
-    const int h = w.h0 + t, r = grp * 32 + lane;
-    // segments (chunk, half) of chunks 0 and last: reference and total
-    float m[2][2], tot[2][2];
-#pragma unroll
-    for (int c = 0; c < 2; ++c)
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const int ch = c ? last : 0;
-        const size_t ci = (((size_t)h * nch + ch) * 2 + hf) * kB + r;
-        m[c][hf] = __ldcg(a.chunk_max + ci);
-        tot[c][hf] = (c == 1 && last == 0) ? 0.f : __ldcg(a.chunk_tot + ci);  // one chunk: count once
-      }
-    float M = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < 2; ++c)
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) M = fmaxf(M, m[c][hf]);
-    float Z = 0.f, A = 0.f;
-#pragma unroll
-    for (int c = 0; c < 2; ++c)
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) Z += tot[c][hf] * exp2f(m[c][hf] - M);
-#pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      const float2 p0 = __ldcg(a.part + ((size_t)h * nb * 2 + hf) * kB + r);  // block 0
-      A += (p0.x + p0.y) * exp2f(m[0][hf] - M);
-      if (nb > 1) {
-        const float2 pl = __ldcg(a.part + (((size_t)h * nb + nb - 1) * 2 + hf) * kB + r);
-        A += (pl.x + pl.y) * exp2f(m[1][hf] - M);
-      }
-      if (s.n % kB != 0 && nb >= 3) {
-        // the last 128 keys reach into block N_b-2 (its columns from t_last on), which lies in
-        // the last chunk or in chunk 0
-        const int cb = (nb - 2) / kProxyChunk;
-        if (cb == last || cb == 0)
-          A += __ldcg(a.rec_extra + ((size_t)h * 2 + hf) * kB + r) * exp2f(m[cb == last ? 1 : 0][hf] - M);
-      }
-    }
-    float c_row = Z > 0.f ? A / Z : 1.f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) c_row += __shfl_xor_sync(0xffffffffu, c_row, o);
-    if (lane == 0) sm.hint_part[t][grp] = c_row;
-  }
-  named_bar_sync(1, SOFTMAX_WARPS * 32);
-  if (threadIdx.x < w.ntiles) {
-    const int t2 = threadIdx.x, h = w.h0 + t2;
-    const float c_bound = (sm.hint_part[t2][0] + sm.hint_part[t2][1] + sm.hint_part[t2][2] + sm.hint_part[t2][3]) *
-                          (1.f / kB);
-    a.hint[h] = (a.route_rule == 0 && c_bound < a.tau) ? 1u : 0u;
-    __threadfence();
-    atomicExch(a.hint_ready + h, 1u);
-  }
-}
-
-// Q_bar pooling CTAs: pooling item i = (head, run of 16 query blocks), CTA p of P taking items
-// p, p+P, ... A producer thread waits (bounded) for the head's hint and, for a hinted head, loads
-// the run's Q blocks by TMA through POOL_STAGES stages laid over the q and k buffers; the 16
-// softmax-sized warps sum each block's rows (32 row groups of 4 rows, one 16-byte chunk of 8
-// columns per thread, then the 32 partial sums per column), take the mean and store it as three
-// bf16 terms, and count the run in pooled_cnt[head]. A head whose hint never came, or came 0, is
-// left to the Q_bar kernel after routing.
-constexpr unsigned long long kHintWaitNs = 4000000ull;  // 4 ms
-__device__ void pool_q_blocks(ProxySmem& sm, const CUtensorMap& q_map, const SelectArgs& a, int p, int P, int warp,
-                              int lane) {
-  const Shape& s = a.s;
-  const int ipr = (s.nb + kProxyChunk - 1) / kProxyChunk;  // runs of 16 query blocks per head
-  const int n_pool_items = s.h_q * ipr;
-  uint8_t* stage0 = reinterpret_cast<uint8_t*>(&sm.q[0][0]);
-  if (warp == PRODUCER_WARP) {
-    if (lane == 0) {
-      tma_prefetch_desc(&q_map);
-      int st = 0, given_up = -1;  // a head whose hint did not come in time is not waited for again
-      for (int pi = p; pi < n_pool_items; pi += P) {
-        const int h = pi / ipr, run = pi % ipr;
-        if (h == given_up) continue;
-        volatile uint32_t* ready = a.hint_ready + h;
-        const unsigned long long t0 = global_ns();
-        bool have = true;
-        while (*ready == 0u) {
-          if (global_ns() - t0 > kHintWaitNs || *reinterpret_cast<volatile int*>(&sm.abort)) {
-            have = false;
-            given_up = h;
-            break;
-          }
-          __nanosleep(256);
-        }
-        if (!have || *reinterpret_cast<volatile uint32_t*>(a.hint + h) == 0u) continue;
-        for (int qb = run * kProxyChunk; qb < min(s.nb, (run + 1) * kProxyChunk); ++qb, ++st) {
-          const int sg = st % POOL_STAGES;
-          if (!mbar_wait(&sm.pool_empty[sg], ((st / POOL_STAGES) & 1) ^ 1, nullptr)) {
-            fail(sm, a.status);
-            break;
-          }
-          sm.stage_info[sg] = h * 65536 + qb;
-          uint8_t* dst = stage0 + (size_t)sg * TILE_BYTES;
-          mbar_arrive_expect_tx(&sm.pool_full[sg], TILE_BYTES);
-          tma_load_3d(&q_map, &sm.pool_full[sg], dst, 0, qb * kB, h);
-          tma_load_3d(&q_map, &sm.pool_full[sg], dst + HALF_BYTES, 64, qb * kB, h);
-        }
-      }
-      // end marker: a plain arrival completes the stage's phase with no bytes
-      const int sg = st % POOL_STAGES;
-      if (mbar_wait(&sm.pool_empty[sg], ((st / POOL_STAGES) & 1) ^ 1, nullptr)) {
-        sm.stage_info[sg] = -1;
-        mbar_arrive(&sm.pool_full[sg]);
-      } else {
-        fail(sm, a.status);
-      }
-    }
-    __syncwarp();
-  } else if (warp < SOFTMAX_WARPS) {
-    const int tid = threadIdx.x;  // 0..511
-    const int cc = tid & 15, rg = tid >> 4;  // 8-column chunk, group of 4 rows
-    const int half = cc >> 3, ch = cc & 7;
-    for (int st = 0;; ++st) {
-      const int sg = st % POOL_STAGES;
-      if (!warp_wait(&sm.pool_full[sg], (st / POOL_STAGES) & 1, &sm.abort)) {
-        fail(sm, a.status);
-        break;
-      }
-      const int info = sm.stage_info[sg];
-      if (info < 0) break;
-      const int h = info >> 16, qb = info & 0xffff;
-      const uint8_t* base = stage0 + (size_t)sg * TILE_BYTES + half * HALF_BYTES;
-      float acc[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-      uint4 u[4];
-#pragma unroll
-      for (int x = 0; x < 4; ++x) u[x] = *reinterpret_cast<const uint4*>(base + sw128_offset(rg * 4 + x, ch));
-#pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&u[x]);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 f = __bfloat1622float2(p2[i]);
-          acc[2 * i] += f.x;
-          acc[2 * i + 1] += f.y;
-        }
-      }
-      float* red = &sm.red[st & 1][0][0];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) red[rg * kD + cc * 8 + i] = acc[i];
-      named_bar_sync(2, SOFTMAX_WARPS * 32);
-      if (tid == 0) mbar_arrive(&sm.pool_empty[sg]);  // every thread has read the stage
-      if (tid < kD) {
-        float v = 0.f;
-#pragma unroll 8
-        for (int g = 0; g < 32; ++g) v += red[g * kD + tid];
-        const int rows = min(kB, s.n - qb * kB);  // a partial last block has fewer rows
-        v *= 1.f / (float)rows;
-        const __nv_bfloat16 b0 = __float2bfloat16_rn(v);
-        const float r1 = v - __bfloat162float(b0);
-        const __nv_bfloat16 b1 = __float2bfloat16_rn(r1);
-        const __nv_bfloat16 b2 = __float2bfloat16_rn(r1 - __bfloat162float(b1));
-        __nv_bfloat16* dst = a.qparts + ((size_t)h * 3 * s.nb + qb) * kD + tid;  // [h][term][nb][128]
-        dst[0] = b0;
-        dst[(size_t)s.nb * kD] = b1;
-        dst[(size_t)2 * s.nb * kD] = b2;
-        const int run_end = min(s.nb, (qb / kProxyChunk + 1) * kProxyChunk);
-        if (tid == 0 && qb == run_end - 1) atomicAdd(a.pooled_cnt + h, 1u);
-      }
-    }
-  }
-}
-
 // RAGGED: n is not a multiple of 128 (separate instance, so the common case keeps the lane-aligned
 // split with no extra work in its exponential loop).
 template <bool RAGGED>
@@ -419,11 +198,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const Shape& s = a.s;
   const int ppg = (s.G + 1) / 2;
-  const int n_proxy = a.proxy_ctas;
-  const bool pooler = (int)blockIdx.x >= n_proxy;
-  const Sched sched(s, n_proxy, (int)gridDim.x > n_proxy);
+  const Sched sched(s, (int)gridDim.x);
   const int cta = blockIdx.x;
-  const int my_items = pooler ? 0 : sched.count(cta);
+  const int my_items = sched.count(cta);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
@@ -440,10 +217,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_init(&sm.s_free[t][b], 8);  // the tile's eight softmax warps
       }
     mbar_init(&sm.mma_done, 1);
-    for (int i = 0; i < POOL_STAGES; ++i) {
-      mbar_init(&sm.pool_full[i], 1);
-      mbar_init(&sm.pool_empty[i], 1);
-    }
     sm.abort = 0;
     fence_mbar_init();
   }
@@ -457,9 +230,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  if (pooler) {
-    pool_q_blocks(sm, q_map, a, cta - n_proxy, (int)gridDim.x - n_proxy, warp, lane);
-  } else if (warp == PRODUCER_WARP) {
+  if (warp == PRODUCER_WARP) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&q_map);
@@ -681,8 +452,6 @@ __global__ void __launch_bounds__(THREADS, 1)
           a.rec_extra[((size_t)h * 2 + half) * kB + r] = rec;
       }
       }
-      // every softmax warp takes part, whether or not its tile had a head or an error occurred
-      if (sched.is_anchor(cta, it)) anchor_done(sm, a, w, sched.apc, t, half, grp, lane);
     }
     __syncwarp();
   } else if (warp >= POOL_WARP) {
@@ -790,6 +559,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
+}  // namespace
+
 int num_sms() {
   static int n = [] {
     int dev = 0, v = 0;
@@ -800,8 +571,6 @@ int num_sms() {
   return n;
 }
 
-}  // namespace
-
 cudaError_t launch_proxy_pass(const CUtensorMap& q_map, const CUtensorMap& k_map, const SelectArgs& a,
                               cudaStream_t st) {
   const size_t smem = sizeof(ProxySmem) + 1024;
@@ -809,22 +578,9 @@ cudaError_t launch_proxy_pass(const CUtensorMap& q_map, const CUtensorMap& k_map
   auto kernel = ragged ? proxy_pass_kernel<true> : proxy_pass_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  // Persistent: one CTA per SM. With the C_struct router a share of the SMs pools Q_bar of the
-  // heads the anchor chunks already show to be Pooled-Estimation, while the rest run the proxy
-  // items; the anchor items go first so the hints come early.
-  const int pairs = a.s.h_kv * ((a.s.G + 1) / 2);
-  const int n_items = pairs * a.s.n_chunks;
-  const int n_anchor = pairs * min(2, a.s.n_chunks);
-  const int sms = num_sms();
-  int n_pool = a.route_rule == 0 ? (sms * kPoolShareNum) / kPoolShareDen : 0;
-  int n_proxy = min(n_items, sms - n_pool);
-  if (n_anchor > n_proxy || n_pool <= 0) {
-    n_pool = 0;
-    n_proxy = min(n_items, sms);
-  }
-  SelectArgs args = a;
-  args.proxy_ctas = n_proxy;
-  kernel<<<n_proxy + n_pool, THREADS, smem, st>>>(q_map, k_map, args);
+  // Persistent: one CTA per SM.
+  const int n_items = a.s.h_kv * ((a.s.G + 1) / 2) * a.s.n_chunks;
+  kernel<<<min(n_items, num_sms()), THREADS, smem, st>>>(q_map, k_map, a);
   return cudaGetLastError();
 }
 

@@ -443,34 +443,23 @@ __global__ void __launch_bounds__(THREADS) mass_route_kernel(const SelectArgs a)
     w_s[i / kB][i % kB] = a.row_w[((size_t)h * nseg + 2 * c0) * kB + i];
   __syncthreads();
   const int t_last = s.n - (nb - 1) * kB;
-  // each warp's key blocks kb0 + warp + 16 i, two at a time with both blocks' sums loaded
-  // before the first is used
-  for (int k0 = 0; k0 < MASS_BLOCKS / NWARP; k0 += 2) {
-  float2 vv[2][2 * kB / 32];
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int kb = kb0 + warp + NWARP * (k0 + k);
-#pragma unroll
-    for (int i = 0; i < 2 * kB / 32; ++i)
-      vv[k][i] = kb < nb ? a.part[(size_t)(h * nb + kb) * 2 * kB + lane + 32 * i] : make_float2(0.f, 0.f);
-  }
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int kb = kb0 + warp + NWARP * (k0 + k);
-    if (kb >= nb) break;
+  for (int kb = kb0 + warp; kb < min(nb, kb0 + MASS_BLOCKS); kb += NWARP) {
+    const float2* v = a.part + (size_t)(h * nb + kb) * 2 * kB + lane;  // [half][128], this lane's rows
     const float* wc = w_s[2 * (kb / kProxyChunk - c0)];         // [half][128]
     double loA = 0.0, hiA = 0.0, loB = 0.0, hiB = 0.0;
-    const float2* v = vv[k];
+    float2 vv[2 * kB / 32];
+#pragma unroll
+    for (int i = 0; i < 2 * kB / 32; ++i) vv[i] = v[32 * i];
 #pragma unroll
     for (int i = 0; i < 2 * kB / 32; ++i) {
       const int r = (lane + 32 * i) & (kB - 1);
       const double ww = wc[lane + 32 * i];
       if (t_last + r >= kB) {
-        loA += (double)v[i].x * ww;
-        hiA += (double)v[i].y * ww;
+        loA += (double)vv[i].x * ww;
+        hiA += (double)vv[i].y * ww;
       } else {
-        loB += (double)v[i].x * ww;
-        hiB += (double)v[i].y * ww;
+        loB += (double)vv[i].x * ww;
+        hiB += (double)vv[i].y * ww;
       }
     }
 #pragma unroll
@@ -489,7 +478,6 @@ __global__ void __launch_bounds__(THREADS) mass_route_kernel(const SelectArgs a)
       if (nb - 3 - kb >= 0) a.ps_x[base + nb - 3 - kb] = hiB;
       else a.ps_x[base + (nb - 3 - kb == -1 ? nb - 2 : nb - 1)] = 0.0;  // kb = N_b-2, N_b-1
     }
-  }
   }
   // the head's last CTA routes it (counter back to zero for the radix levels that reuse it)
   __threadfence();

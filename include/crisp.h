@@ -199,7 +199,10 @@ int crisp_selftest_timeout(void* ws, size_t ws_bytes, uint64_t limit_ns, void* s
  *     it until the process exits). Shapes whose workspace (crisp_workspace_size) exceeds 32 MiB
  *     return CRISP_ERR_WORKSPACE without launching anything.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
- *     that device current; make that first call before any stream capture.
+ *     that device current; make that first call before any stream capture. The address is kept
+ *     for the life of the process: after cudaDeviceReset the library's module is loaded again
+ *     and the kept address is stale, so a process that resets a device must not call this entry
+ *     point on that device afterwards.
  *   - All calls share the array and it keeps the last call's contents; the call clears what must
  *     start at zero. Calls that overlap on the GPU (other streams, other threads) race on it.
  *   - device_status: NULL, or a device int the caller has zeroed; a device-side failure stores its
