@@ -33,9 +33,9 @@ from dynamic_block_sparse_proxy_b200 import workloads as W  # noqa: E402
 
 METRIC = "prefill tokens/s per layer (select+sparse attn) at 128k; % bf16 peak, % HBM BW"
 DEFAULT_WORKLOAD = "llama8b_128k"
-# kernels per step: proxy pass, routing, 5 for the PE path (Q_bar, scores, row softmax, two
-# histogram levels), 3 for the merge, attention
-KERNELS_PER_STEP = 11
+# kernels per step: proxy pass, 2 for routing (row statistics, block masses + route), 5 for the PE
+# path (Q_bar, scores, row softmax, two histogram levels), 3 for the merge, attention
+KERNELS_PER_STEP = 12
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
