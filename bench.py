@@ -132,21 +132,38 @@ def select_bytes(w, n_pe_heads: int, total_pairs: int) -> float:
     return float(k_bytes + qlast + qpe + idx)
 
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attention launch on the 128k
-# workload, from a one-pass ncu capture of this command's own launch. The figure belongs to the
-# kernel source it was taken on; for any other source or workload the bench reports null.
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attention launch, and the sum
+# over the selection kernels of one step, on the 128k workload, from a three-metric ncu capture
+# of this command's own timed step. Each figure belongs to the kernel sources it was taken on
+# (SHA-256 of the source, or of the selection sources in order); for any other source or workload
+# the bench reports null.
 ATTN_TRAFFIC = {"workload": "llama8b_128k",
-                "source_sha256": "7d0a430321f4f231d5978bce192dbc519320892784022e99096184bcd0f21f1a",
-                "bytes": 2.66e9 + 1.06e9}
+                "source_sha256": "93b54c6d7a93267e496f992d9f9bfeb5b74ee88130a05536d16d3d9c7ab6aecc",
+                "bytes": 2.70141e9 + 1.05458e9}
+SELECT_SOURCES = ["proxy_pass.cu", "route_threshold.cu", "pe_cut.cu", "merge.cu", "sm100.cuh", "crisp_internal.h"]
+SELECT_TRAFFIC = {"workload": "llama8b_128k",
+                  "source_sha256": "a3fb6ff3c0cc4cba9d7ef1208527e3eb96720cf24a7bf2c30e90facd62b679cf",
+                  "bytes": 1282.31e6 + 86.82e6}
+
+
+def _sources_sha(names):
+    h = hashlib.sha256()
+    for name in names:
+        with open(os.path.join(ROOT, "dynamic_block_sparse_proxy_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 def attn_traffic(w):
-    src = os.path.join(ROOT, "dynamic_block_sparse_proxy_b200", "csrc", "sparse_attn.cu")
-    with open(src, "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()
-    if w.name != ATTN_TRAFFIC["workload"] or sha != ATTN_TRAFFIC["source_sha256"]:
+    if w.name != ATTN_TRAFFIC["workload"] or _sources_sha(["sparse_attn.cu"]) != ATTN_TRAFFIC["source_sha256"]:
         return None
     return ATTN_TRAFFIC["bytes"]
+
+
+def select_traffic(w):
+    if w.name != SELECT_TRAFFIC["workload"] or _sources_sha(SELECT_SOURCES) != SELECT_TRAFFIC["source_sha256"]:
+        return None
+    return SELECT_TRAFFIC["bytes"]
 
 
 # Index-selection rules: CRISP's own (default), the FlexPrefill baseline the CRISP paper compares
@@ -313,7 +330,7 @@ def run_crisp(args):
                      "density": total_pairs / dense_pairs},
         "select_roofline": {"bound": "hbm", "achieved": sel_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                             "frac": sel_gbs / pk["hbm_gbs"], "bytes_per_launch": sb,
-                            "ms": mean_sel * 1e3, "pe_heads": n_pe},
+                            "traffic": select_traffic(w), "ms": mean_sel * 1e3, "pe_heads": n_pe},
         "attn_ms": mean_att * 1e3,
         "select_ms": mean_sel * 1e3,
         "e2e": e2e,

@@ -316,11 +316,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int st = step % NSK;
         const int prev_vs = (step + NSV - 1) % NSV;
         if (step > 0) {
-          // V of the previous step: O_t += P_t V (P_t sits in the S_t columns), or skip it
+          // V of the previous step: O_t += P_t V (P_t sits in the S_t columns), or skip it. V is
+          // waited for first (it is normally in long before P), so the MMAs go out as soon as P is.
           trace_mark(a.trace, 0, role, 3, step);
           const bool use = (prev_mask & bit) != 0;
-          if ((use && !mbar_wait(&sm.p_full[t], pv_n & 1, abort)) ||
-              !mbar_wait(&sm.v_full[prev_vs], ((step - 1) / NSV) & 1, abort)) {
+          if (!mbar_wait(&sm.v_full[prev_vs], ((step - 1) / NSV) & 1, abort) ||
+              (use && !mbar_wait(&sm.p_full[t], pv_n & 1, abort))) {
             fail(sm, a.status, CRISP_ERR_DEVICE_TIMEOUT);
             break;
           }
