@@ -322,10 +322,13 @@ def run_crisp(args):
         "dtype": "bf16",
         "data": "synthetic (seeded planted-structure generator)",
         "config": bench_config(w, args, world),
+        # The attention launch lasts tens of milliseconds and the timed region well under a
+        # second, at clocks near the maximum: the burst figure is the denominator, and the
+        # sustained one (a seconds-long GEMM loop at a lower clock under the power cap) is beside it.
         "roofline": {"bound": "tensor", "kernel": "sparse_attn", "achieved": achieved_tf,
-                     "peak": sustained, "unit": "TFLOP/s", "frac": achieved_tf / sustained,
-                     "peak_kind": f"bf16 sustained ({src})",
-                     "frac_of_burst": achieved_tf / pk["bf16_tflops"], "traffic": attn_traffic(w),
+                     "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved_tf / pk["bf16_tflops"],
+                     "peak_kind": f"bf16 burst ({src})",
+                     "frac_of_sustained": achieved_tf / sustained, "traffic": attn_traffic(w),
                      "flops_per_launch": fl, "selected_pairs": total_pairs,
                      "density": total_pairs / dense_pairs},
         "select_roofline": {"bound": "hbm", "achieved": sel_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
