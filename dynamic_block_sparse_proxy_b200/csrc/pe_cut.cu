@@ -212,20 +212,10 @@ __global__ void __launch_bounds__(SC_THREADS) scores_kernel(const __grid_constan
 
 // ------------------------------------------------------------------------ histograms, select
 // Histogram masses are fixed point (2^-40 units, rounded to nearest, ties to even): integer
-// atomics are exact and order-independent, and N_b * 2^40 stays far below 2^64. For p >= 0 with
-// biased exponent e and 24-bit significand s, p * 2^40 = s * 2^(e - 110): a shift of s, rounded
-// when it runs right, all in integer arithmetic.
+// atomics are exact and order-independent, and N_b * 2^40 stays far below 2^64. The product
+// p * 2^40 of an fp32 p is exact in fp64, so one conversion rounds it as the definition asks.
 __device__ __forceinline__ unsigned long long to_fixed(float p) {
-  const uint32_t bits = __float_as_uint(p);
-  const int e = (int)(bits >> 23);
-  if (e == 0) return 0ull;  // zero, or below 2^-126: rounds to 0
-  const unsigned long long sig = (bits & 0x7fffffu) | 0x800000u;
-  const int sh = e - 110;
-  if (sh >= 0) return sig << sh;
-  const int k = -sh;
-  if (k > 25) return 0ull;
-  const unsigned long long q = sig >> k, rem = sig & ((1ull << k) - 1ull), half = 1ull << (k - 1);
-  return q + ((rem > half || (rem == half && (q & 1ull))) ? 1ull : 0ull);
+  return __double2ull_rn((double)p * kMassUnit);  // exact product, rounded to nearest even
 }
 
 // Level-1 histogram of one row step (all lanes call it): only the mass of a bin decides the
@@ -234,9 +224,14 @@ __device__ __forceinline__ unsigned long long to_fixed(float p) {
 // as three 16-bit parts (redux.sync, one instruction per part for every group at once) and its
 // lowest lane adds them to three 32-bit shared arrays: no 64-bit shared atomics, and no two lanes
 // of a warp hit the same word. A CTA's part sums stay below 2^32 (at most 8192 entries of < 2^16).
-__device__ __forceinline__ void warp_mass_add(uint32_t (*smass3)[kHistBins], bool valid, float p) {
+// Only bins [kL1Lo, kL1Lo + kL1Bins) can receive mass: an entry with a non-zero fixed-point mass has
+// p >= 2^-41 (biased exponent >= 86, bin >= 86 * 8), and p <= 1 up to rounding (bin <= 127 * 8).
+constexpr uint32_t kL1Lo = 86u * 8u;
+constexpr uint32_t kL1Bins = 336;
+__device__ __forceinline__ void warp_mass_add(uint32_t (*smass3)[kL1Bins], bool valid, float p) {
   const unsigned long long fx = valid ? to_fixed(p) : 0ull;
-  const uint32_t key = fx != 0ull ? (__float_as_uint(p) >> 20) : 0xffffffffu;
+  const uint32_t bin = (__float_as_uint(p) >> 20) - kL1Lo;
+  const uint32_t key = (fx != 0ull && bin < kL1Bins) ? bin : 0xffffffffu;
   const unsigned grp = __match_any_sync(0xffffffffu, key);
   const uint32_t s0 = __reduce_add_sync(grp, (uint32_t)(fx & 0xffffu));
   const uint32_t s1 = __reduce_add_sync(grp, (uint32_t)((fx >> 16) & 0xffffu));
@@ -393,8 +388,8 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32, 4) rowsoft_kernel(const Sel
   const int h = blockIdx.y;
   if (!is_pe(a, h)) return;
   const Shape& s = a.s;
-  __shared__ uint32_t smass3[3][kHistBins];  // 16-bit parts of the fixed-point bin masses
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) smass3[0][i] = smass3[1][i] = smass3[2][i] = 0u;
+  __shared__ uint32_t smass3[3][kL1Bins];  // 16-bit parts of the fixed-point bin masses
+  for (int i = threadIdx.x; i < (int)kL1Bins; i += blockDim.x) smass3[0][i] = smass3[1][i] = smass3[2][i] = 0u;
   __syncthreads();
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int qb = blockIdx.x * ROWS_PER_CTA + w;
@@ -428,12 +423,15 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32, 4) rowsoft_kernel(const Sel
       const float inv = 1.f / z;
 #pragma unroll
       for (int u = 0; u < 32; ++u) {
-        if (u * 32 < L) {
-          const int i = u * 32 + lane;
-          const float p = x[u] * inv;
-          if (i < L) row[i] = p;
-          warp_mass_add(smass3, i < L, p);
-        }
+        const int i = u * 32 + lane;
+        if (u * 32 < L && i < L) row[i] = x[u] * inv;
+      }
+      // the histogram from the values just stored (this thread's own stores), in a rolled loop
+#pragma unroll 2
+      for (int base = 0; base < L; base += 32) {
+        const int i = base + lane;
+        const float p = i < L ? row[i] : 0.f;
+        warp_mass_add(smass3, i < L, p);
       }
     } else {
       float mx = -INFINITY;
@@ -489,10 +487,10 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32, 4) rowsoft_kernel(const Sel
   }
   __syncthreads();
   // the CTA's bin masses (the parts recombined), then its share of the global histogram
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) {
+  for (int i = threadIdx.x; i < (int)kL1Bins; i += blockDim.x) {
     const unsigned long long m = (unsigned long long)smass3[0][i] + ((unsigned long long)smass3[1][i] << 16) +
                                  ((unsigned long long)smass3[2][i] << 32);
-    if (m) atomicAdd(a.hist_mass + (size_t)h * kHistBins + i, m);
+    if (m) atomicAdd(a.hist_mass + (size_t)h * kHistBins + kL1Lo + i, m);
   }
   if (flush_and_check_last(a, h, nullptr, nullptr, 0, gridDim.x)) select_bin(a, h, 1);
 }
