@@ -142,8 +142,8 @@ ATTN_TRAFFIC = {"workload": "llama8b_128k",
                 "bytes": 2.70141e9 + 1.05458e9}
 SELECT_SOURCES = ["proxy_pass.cu", "route_threshold.cu", "pe_cut.cu", "merge.cu", "sm100.cuh", "crisp_internal.h"]
 SELECT_TRAFFIC = {"workload": "llama8b_128k",
-                  "source_sha256": "a3fb6ff3c0cc4cba9d7ef1208527e3eb96720cf24a7bf2c30e90facd62b679cf",
-                  "bytes": 1282.31e6 + 86.82e6}
+                  "source_sha256": "e3c89aa9147e72fb8b5898aaaf057e16f3f2b5184f129b8756dd27bd55ae5b80",
+                  "bytes": 1283.68e6 + 88.04e6}
 
 
 def _sources_sha(names):
@@ -291,7 +291,7 @@ def run_crisp(args):
 
     e2e = None
     if args.e2e:
-        e2e = e2e_pipelined(w, q, k, v, params, idx, ws, max(2, min(args.steps, 4)), dev, stream)
+        e2e = e2e_pipelined(w, q, k, v, params, idx, ws, max(4, min(args.steps, 8)), dev, stream)
         e2e_s = max_over_ranks(e2e.pop("seconds_per_step"), world, dev)
         e2e.update(value=job_tokens_per_s(world, w.n, 1, e2e_s), ms_per_step=e2e_s * 1e3)
 
@@ -359,8 +359,10 @@ def e2e_pipelined(w, q, k, v, params, idx, ws, steps: int, dev, stream) -> dict:
     and V from pinned host memory, selects (crisp.select), attends one kv-group at a time
     (crisp.sparse_prefill on the group's heads and index rows) and copies each group's output back
     to pinned host memory as soon as that group is done. Two sets of device inputs and outputs let
-    step i+1's uploads run during step i's attention, as a prefill pipeline over layers would; one
-    warm-up step, then `steps` timed steps from the first upload to the last download."""
+    step i+1's uploads run during step i's attention, as a prefill pipeline over layers would. One
+    warm-up step runs to completion first; the timed region then covers `steps` steps from the
+    first step's upload (nothing else running) to the last step's download, so every timed step's
+    copies lie inside it and the pipeline fills once."""
     G = w.h_q // w.h_kv
     qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
     oh = [torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(2)]
@@ -381,6 +383,7 @@ def e2e_pipelined(w, q, k, v, params, idx, ws, steps: int, dev, stream) -> dict:
     for i in range(total):
         b = i % 2
         if i == 1:
+            torch.cuda.synchronize()  # the warm-up step is done
             t0.record(up)  # timed region starts with step 1's first upload
         with torch.cuda.stream(up):
             if in_free[b] is not None:
