@@ -288,6 +288,7 @@ def run_crisp(args):
                  "dense_tflops": attn_flops(w.h_q * nb * (nb + 1) // 2, w.d) / dense_s / 1e12,
                  "steps": args.dense_steps, "clocks": clocks_d}
         del od, lsed
+        dense["torch_sdpa"] = torch_sdpa_reference(q, k, v, w, nb, args.dense_steps, flush, stream)
 
     e2e = None
     if args.e2e:
@@ -354,6 +355,30 @@ def run_crisp(args):
 
 
 # ---------------------------------------------------------------------------- end to end
+def torch_sdpa_reference(q, k, v, w, nb, steps: int, flush, stream) -> dict:
+    """An outside reference for the dense number: PyTorch's own causal scaled-dot-product attention
+    (whichever backend it picks) on the same inputs, timed like the dense leg. FLOPs are counted as
+    for the dense leg (full diagonal tiles), so the two TFLOP/s figures compare directly."""
+    import torch.nn.functional as F
+    try:
+        qs, ks, vs = q.unsqueeze(0), k.unsqueeze(0), v.unsqueeze(0)
+        with torch.cuda.stream(stream):
+            F.scaled_dot_product_attention(qs, ks, vs, is_causal=True, enable_gqa=True)
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+            torch.cuda.synchronize()
+            for e0, e1 in ev:
+                flush.fill_(5)
+                e0.record(stream)
+                F.scaled_dot_product_attention(qs, ks, vs, is_causal=True, enable_gqa=True)
+                e1.record(stream)
+            torch.cuda.synchronize()
+        sec = float(np.mean([e0.elapsed_time(e1) for e0, e1 in ev])) / 1e3
+        return {"ms": sec * 1e3, "tflops": attn_flops(w.h_q * nb * (nb + 1) // 2, w.d) / sec / 1e12,
+                "call": "torch.nn.functional.scaled_dot_product_attention(is_causal=True, enable_gqa=True)"}
+    except Exception as e:  # a missing backend is reported, not fatal
+        return {"unavailable": f"{type(e).__name__}: {e}"[:200]}
+
+
 def e2e_pipelined(w, q, k, v, params, idx, ws, steps: int, dev, stream) -> dict:
     """The metric end to end through the public API with host buffers: every step copies its Q, K
     and V from pinned host memory, selects (crisp.select), attends one kv-group at a time
