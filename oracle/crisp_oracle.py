@@ -373,3 +373,71 @@ def dense_causal_attention(q, k, v):
     m = s.max(axis=1, keepdims=True)
     e = np.exp(s - m)
     return (e / e.sum(axis=1, keepdims=True)) @ v
+
+
+# ----------------------------------------------------------------------------------------------
+# FP8 variant of the attention logits: Q and K quantised to 8-bit E4M3 per 128-row block
+# (the OCP 8-bit floating-point format: 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits,
+# no infinities, largest finite value 448, subnormals m * 2^-9). The attention itself is then the
+# exact attention of the dequantised Q and K (attention_rows on them).
+# ----------------------------------------------------------------------------------------------
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(code: np.ndarray) -> np.ndarray:
+    """Value of each E4M3 code (uint8); the two NaN codes (0x7f, 0xff) decode to nan."""
+    c = np.asarray(code, dtype=np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((e == 0xF) & (m == 0x7), np.nan, mag)
+    return sign * mag
+
+
+def e4m3_encode(y: np.ndarray) -> np.ndarray:
+    """Round each value to the nearest E4M3 value, ties to the even code, saturating at +-448
+    (finite inputs); the sign bit is the input's, so small negative values give -0 (0x80). Written from the format: the representable magnitudes are enumerated and the
+    nearest one is picked, so no rounding arithmetic can be wrong here."""
+    y = np.asarray(y, dtype=np.float64)
+    codes = np.arange(0x7F, dtype=np.int64)                  # 0x00 .. 0x7e: every finite magnitude
+    mags = e4m3_decode(codes)                                # ascending
+    a = np.minimum(np.abs(y), E4M3_MAX)
+    hi = np.searchsorted(mags, a, side="left").clip(0, len(mags) - 1)
+    lo = (hi - 1).clip(0, None)
+    d_hi = np.abs(mags[hi] - a)
+    d_lo = np.abs(a - mags[lo])
+    pick = np.where(d_lo < d_hi, lo, hi)
+    tie = d_lo == d_hi
+    pick = np.where(tie & (lo != hi), np.where(codes[lo] % 2 == 0, lo, hi), pick)
+    out = codes[pick]
+    out = np.where(np.signbit(y), out | 0x80, out)          # the sign is kept, also on zero
+    return out.astype(np.uint8)
+
+
+def quantize_blocks_fp8(x: np.ndarray, B: int = 128):
+    """Per block of B rows of x [n, d] (bf16 values widened exactly): amax = max |x| in fp32,
+    codes = E4M3(fp32(x) * fp32(448 / amax)) with the product and quotient rounded to fp32, and the
+    dequantisation scale fp32(amax / 448); an all-zero block gets codes 0 and scale 1. Returns
+    (codes uint8 [n, d], scales float32 [N_b]); the dequantised block is e4m3_decode(codes) * scale."""
+    n = x.shape[0]
+    nb = -(-n // B)
+    xs = np.asarray(x, dtype=np.float32)
+    codes = np.zeros(xs.shape, dtype=np.uint8)
+    scales = np.ones(nb, dtype=np.float32)
+    for b in range(nb):
+        blk = xs[b * B:min(n, (b + 1) * B)]
+        amax = np.float32(np.abs(blk).max()) if blk.size else np.float32(0)
+        if amax == 0:
+            continue
+        inv = np.float32(np.float32(E4M3_MAX) / amax)
+        codes[b * B:min(n, (b + 1) * B)] = e4m3_encode((blk * inv).astype(np.float32))
+        scales[b] = np.float32(amax / np.float32(E4M3_MAX))
+    return codes, scales
+
+
+def dequantize_blocks_fp8(codes: np.ndarray, scales: np.ndarray, B: int = 128) -> np.ndarray:
+    """fp64 values of the quantised blocks: e4m3_decode(code) * scale of the row's block."""
+    vals = e4m3_decode(codes)
+    rows = np.arange(codes.shape[0]) // B
+    return vals * np.asarray(scales, dtype=np.float64)[rows][:, None]

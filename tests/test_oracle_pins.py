@@ -539,3 +539,52 @@ def test_pooled_scores_hand_case_catches_plausible_mistakes(monkeypatch, mistake
         g, q, k, _ = _pooled_case()
         got = [[x.tolist() for x in O.pe_select(q, k, g["B"], c["gamma"])[0]] for c in g["cuts"]]
         assert any(gl != c["lists"] for gl, c in zip(got, g["cuts"]))
+
+
+# ---------------------------------------------------------------------------------------------
+# FP8 (E4M3) quantisation of the attention logits' operands
+# ---------------------------------------------------------------------------------------------
+def test_e4m3_codes_from_the_format_definition():
+    """Values whose codes follow from the format (bias 7, 3 mantissa bits, subnormals m * 2^-9,
+    largest finite 448), including ties to the even code and saturation."""
+    cases = {1.0: 0x38, 448.0: 0x7E, 0.5: 0x30, 2.0 ** -6: 0x08, 2.0 ** -9: 0x01,
+             1.0625: 0x38,          # halfway between 1.0 (even) and 1.125
+             1.1875: 0x3A,          # halfway between 1.125 and 1.25 (even)
+             500.0: 0x7E, 1e6: 0x7E, -1.0: 0xB8, -448.0: 0xFE,
+             3 * 2.0 ** -10: 0x02,  # halfway between 1 and 2 subnormal units (2 is even)
+             2.0 ** -10: 0x00,      # halfway between 0 (even) and the smallest subnormal
+             2.0 ** -11: 0x00, 240.0: 0x77, 0.0: 0x00}
+    for v, code in cases.items():
+        assert int(O.e4m3_encode(np.float32(v))) == code, (v, hex(int(O.e4m3_encode(np.float32(v)))), hex(code))
+    assert O.e4m3_decode(np.array([0x7E]))[0] == 448.0 and O.e4m3_decode(np.array([0x01]))[0] == 2.0 ** -9
+
+
+def test_e4m3_round_trip_and_library_cast():
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    assert (O.e4m3_encode(O.e4m3_decode(codes)) == codes).all()
+    rng = np.random.default_rng(0)
+    y = np.concatenate([rng.uniform(-448, 448, 20000), rng.normal(0, 1, 20000),
+                        rng.normal(0, 0.01, 20000)]).astype(np.float32)
+    ref = torch.from_numpy(y).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert (O.e4m3_encode(y) == ref).all()
+
+
+def test_quantize_blocks_fp8_properties():
+    rng = np.random.default_rng(1)
+    n, B = 300, 128   # a partial last block
+    x = torch.from_numpy(rng.normal(0, 2, (n, 128))).to(torch.bfloat16).double().numpy()
+    x[128:256] = 0.0  # an all-zero block
+    codes, scales = O.quantize_blocks_fp8(x, B)
+    assert scales[1] == 1.0 and (codes[128:256] == 0).all()
+    deq = O.dequantize_blocks_fp8(codes, scales, B)
+    for b in (0, 2):
+        blk = slice(b * B, min(n, (b + 1) * B))
+        amax = np.abs(x[blk]).max()
+        # the element at the block's amax lands on the largest code
+        i = np.unravel_index(np.abs(x[blk]).argmax(), x[blk].shape)
+        assert (codes[blk][i] & 0x7F) == 0x7E
+        assert scales[b] == np.float32(np.float32(amax) / np.float32(448.0))
+        # every value within half a unit of its binade (2^-4 relative) or of the subnormal step
+        err = np.abs(deq[blk] - x[blk])
+        bound = np.maximum(np.abs(x[blk]) * 2.0 ** -4, 2.0 ** -10 * scales[b]) * (1 + 1e-6)
+        assert (err <= bound).all()
