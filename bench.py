@@ -290,6 +290,33 @@ def run_crisp(args):
         del od, lsed
         dense["torch_sdpa"] = torch_sdpa_reference(q, k, v, w, nb, args.dense_steps, flush, stream)
 
+    # the FP8 variant of the logits on the same inputs and index (after the timed region; the
+    # headline stays bf16): its attention time, including the quantisation of Q and K, and how far
+    # its output lies from the bf16 kernel's
+    fp8 = None
+    if args.fp8:
+        buf = crisp.fp8qk_buffer(w.h_q, w.h_kv, w.n, dev)
+        o8, l8 = torch.empty_like(q), torch.empty_like(lse)
+        crisp.sparse_prefill_fp8qk(q, k, v, idx, o=o8, lse=l8, ws=ws, fp8_buf=buf)
+        f_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.dense_steps)]
+        torch.cuda.synchronize()
+        for e0, e1 in f_ev:
+            flush.fill_(3)
+            e0.record(stream)
+            crisp.sparse_prefill_fp8qk(q, k, v, idx, o=o8, lse=l8, ws=ws, fp8_buf=buf)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        crisp.check_status(ws, "fp8qk")
+        f_s = float(np.mean([e0.elapsed_time(e1) for e0, e1 in f_ev])) / 1e3
+        dev_abs = (o8.float() - o.float()).abs()
+        fp8 = {"attn_ms": f_s * 1e3, "tflops": attn_flops(total_pairs, w.d) / f_s / 1e12,
+               "speedup_vs_bf16": float(t_att.mean()) / f_s, "max_abs_vs_bf16": float(dev_abs.max()),
+               "mean_abs_vs_bf16": float(dev_abs.mean()), "steps": args.dense_steps,
+               "what": "S = Q K^T on E4M3 codes with per-(head, 128-row block) scales; P, V and O as in "
+                       "the bf16 kernel; the time includes quantising Q and K"}
+        del buf, o8, l8, dev_abs
+
     e2e = None
     if args.e2e:
         e2e = e2e_pipelined(w, q, k, v, params, idx, ws, max(4, min(args.steps, 8)), dev, stream)
@@ -338,6 +365,7 @@ def run_crisp(args):
         "attn_ms": mean_att * 1e3,
         "select_ms": mean_sel * 1e3,
         "e2e": e2e,
+        "fp8_qk_variant": fp8,
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": clocks,
     }
@@ -557,6 +585,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--no-fp8", dest="fp8", action="store_false",
+                    help="skip the FP8-logits variant leg (run after the timed region)")
     ap.add_argument("--no-dense", dest="dense", action="store_false",
                     help="skip the dense-attention comparison run after the timed region")
     ap.add_argument("--dense-steps", type=int, default=2)

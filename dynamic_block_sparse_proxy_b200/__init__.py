@@ -23,7 +23,7 @@ STATUS_NAMES = {
 }
 EXPORTED = ["crisp_workspace_size", "crisp_select", "crisp_sparse_prefill", "crisp_prefill",
             "crisp_dense_prefill", "crisp_get_status", "crisp_status_string", "crisp_selftest_timeout",
-            "crisp_select_noalloc", "crisp_prefill_varlen"]
+            "crisp_select_noalloc", "crisp_prefill_varlen", "crisp_fp8qk_buffer_size", "crisp_sparse_prefill_fp8qk"]
 
 
 class CrispError(RuntimeError):
@@ -68,8 +68,12 @@ def lib() -> ctypes.CDLL:
         L.crisp_status_string.argtypes = [i32]
         L.crisp_status_string.restype = ctypes.c_char_p
         L.crisp_selftest_timeout.argtypes = [vp, sz, ctypes.c_uint64, vp]
+        L.crisp_fp8qk_buffer_size.argtypes = [i32, i32, i32, i32]
+        L.crisp_fp8qk_buffer_size.restype = sz
+        L.crisp_sparse_prefill_fp8qk.argtypes = [vp, vp, vp, i32, i32, i32, i32, I, vp, vp, vp, sz, vp, sz, vp]
         for name in ("crisp_select", "crisp_sparse_prefill", "crisp_prefill", "crisp_dense_prefill",
-                     "crisp_get_status", "crisp_selftest_timeout", "crisp_prefill_varlen"):
+                     "crisp_get_status", "crisp_selftest_timeout", "crisp_prefill_varlen",
+                     "crisp_sparse_prefill_fp8qk"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -285,6 +289,50 @@ def dense_prefill(q, k, v, o=None, lse=None, ws=None, want_lse: bool = True):
     return o, lse
 
 
+def fp8qk_buffer(h_q: int, h_kv: int, n: int, device, d: int = 128) -> torch.Tensor:
+    """Device buffer for the E4M3 codes and scales of crisp_sparse_prefill_fp8qk."""
+    nbytes = int(lib().crisp_fp8qk_buffer_size(h_q, h_kv, n, d))
+    if nbytes == 0:
+        raise CrispError(-2, "crisp_fp8qk_buffer_size")
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def fp8qk_views(buf: torch.Tensor, h_q: int, h_kv: int, n: int, d: int = 128):
+    """(Q codes [h_q, n, d] uint8, K codes [h_kv, n, d] uint8, Q scales [h_q, N_b] float32,
+    K scales [h_kv, N_b] float32) inside an fp8qk buffer, in the layout crisp.h documents."""
+    nb = -(-n // 128)
+    offs, off = [], 0
+    for nbytes in (h_q * n * d, h_kv * n * d, h_q * nb * 4, h_kv * nb * 4):
+        offs.append(off)
+        off = -(-(off + nbytes) // 256) * 256
+    q8 = buf[offs[0]:offs[0] + h_q * n * d].view(h_q, n, d)
+    k8 = buf[offs[1]:offs[1] + h_kv * n * d].view(h_kv, n, d)
+    qs = buf[offs[2]:offs[2] + h_q * nb * 4].view(torch.float32).view(h_q, nb)
+    ks = buf[offs[3]:offs[3] + h_kv * nb * 4].view(torch.float32).view(h_kv, nb)
+    return q8, k8, qs, ks
+
+
+def sparse_prefill_fp8qk(q, k, v, index: Index, o=None, lse=None, ws=None, fp8_buf=None, want_lse: bool = True):
+    """Block-sparse causal attention with E4M3 logits (crisp_sparse_prefill_fp8qk): Q and K are
+    quantised per head and 128-row block into fp8_buf, then S = Q K^T runs on the codes.
+    Returns (o, lse, fp8_buf)."""
+    h_q, h_kv, n, d = _qkv_shape(q, k, v)
+    ws = ws if ws is not None else workspace(h_q, h_kv, n, q.device, d)
+    fp8_buf = fp8_buf if fp8_buf is not None else fp8qk_buffer(h_q, h_kv, n, q.device, d)
+    o = o if o is not None else torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(h_q, n, device=q.device, dtype=torch.float32)
+    _check_out(q, o, lse)
+    index.check(h_q, n, need_select_fields=False)
+    ix = index.c()
+    _check(lib().crisp_sparse_prefill_fp8qk(q.data_ptr(), k.data_ptr(), v.data_ptr(), h_q, h_kv, n, d,
+                                            ctypes.byref(ix), o.data_ptr(),
+                                            lse.data_ptr() if lse is not None else None, ws.data_ptr(),
+                                            ws.numel(), fp8_buf.data_ptr(), fp8_buf.numel(), _stream(q)),
+           "crisp_sparse_prefill_fp8qk")
+    return o, lse, fp8_buf
+
+
 def get_status(ws: torch.Tensor) -> int:
     """Synchronise the current stream and return (and clear) the device status word."""
     return int(lib().crisp_get_status(ws.data_ptr(), _stream(ws)))
@@ -301,5 +349,6 @@ def selftest_timeout(ws: torch.Tensor, limit_ns: int) -> int:
 
 
 __all__ = ["Params", "Index", "CrispError", "lib", "workspace_size", "workspace", "select", "sparse_prefill",
-           "prefill", "dense_prefill", "get_status", "check_status", "selftest_timeout",
+           "prefill", "dense_prefill", "get_status", "check_status", "selftest_timeout", "fp8qk_buffer",
+           "fp8qk_views", "sparse_prefill_fp8qk",
            "EXPORTED", "LIB_PATH"]

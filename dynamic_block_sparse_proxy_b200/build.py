@@ -14,7 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libcrisp.so")
 SOURCES = ["crisp_api.cu", "proxy_pass.cu", "route_threshold.cu", "pe_cut.cu", "merge.cu", "sparse_attn.cu",
-           "noalloc.cu"]
+           "noalloc.cu", "fp8_qk.cu"]
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
          "-Xcompiler", "-fPIC", "-Xcompiler", "-O3"]
 

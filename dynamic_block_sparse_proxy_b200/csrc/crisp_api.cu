@@ -329,6 +329,94 @@ int crisp_prefill_varlen(const void* q, const void* k, const void* v, int h_q, i
   return CRISP_OK;
 }
 
+namespace {
+
+struct Fp8Layout {
+  size_t q8, k8, qs, ks, total;
+};
+
+Fp8Layout fp8_layout(const Shape& s) {
+  Fp8Layout f{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  f.q8 = take((size_t)s.h_q * s.n * kD);
+  f.k8 = take((size_t)s.h_kv * s.n * kD);
+  f.qs = take((size_t)s.h_q * s.nb * 4);
+  f.ks = take((size_t)s.h_kv * s.nb * 4);
+  f.total = off;
+  return f;
+}
+
+// 3D uint8 view [heads][n][128] of E4M3 codes with 128x128x1 boxes (one 128-byte swizzle span per
+// row): rows past n read as zeros.
+int make_map3_u8(CUtensorMap* m, const void* base, uint64_t n, uint64_t heads) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return CRISP_ERR_CUDA;
+  cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)n, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)kD, (cuuint64_t)kD * n};
+  cuuint32_t box[3] = {(cuuint32_t)kD, (cuuint32_t)kB, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? CRISP_OK : CRISP_ERR_CUDA;
+}
+
+}  // namespace
+
+size_t crisp_fp8qk_buffer_size(int h_q, int h_kv, int n, int d) {
+  Shape s;
+  if (check_shape(h_q, h_kv, n, d, &s) != CRISP_OK) return 0;
+  return fp8_layout(s).total;
+}
+
+int crisp_sparse_prefill_fp8qk(const void* q, const void* k, const void* v, int h_q, int h_kv, int n, int d,
+                               const crisp_index* idx, void* o, float* lse, void* ws, size_t ws_bytes,
+                               void* fp8_buf, size_t fp8_bytes, void* stream) {
+  Shape s;
+  int rc = check_shape(h_q, h_kv, n, d, &s);
+  if (rc == CRISP_OK && (!tensors_ok(q, k, v) || v == nullptr || o == nullptr || !aligned(o, 16)))
+    rc = CRISP_ERR_INVALID_ARG;
+  if (rc == CRISP_OK) rc = check_index(idx, false);
+  if (rc == CRISP_OK) rc = check_ws(ws, ws_bytes, s);
+  if (rc == CRISP_OK && (fp8_buf == nullptr || !aligned(fp8_buf, 256))) rc = CRISP_ERR_INVALID_ARG;
+  if (rc == CRISP_OK && fp8_bytes < fp8_layout(s).total) rc = CRISP_ERR_WORKSPACE;
+  if (rc != CRISP_OK) return rc;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Fp8Layout f = fp8_layout(s);
+  uint8_t* q8 = at<uint8_t>(fp8_buf, f.q8);
+  uint8_t* k8 = at<uint8_t>(fp8_buf, f.k8);
+  float* qs = at<float>(fp8_buf, f.qs);
+  float* ks = at<float>(fp8_buf, f.ks);
+  if (launch_fp8_quant(static_cast<const __nv_bfloat16*>(q), s.h_q, s.n, s.ld, q8, qs, st) != cudaSuccess ||
+      launch_fp8_quant(static_cast<const __nv_bfloat16*>(k), s.h_kv, s.n, s.ld, k8, ks, st) != cudaSuccess)
+    return CRISP_ERR_CUDA;
+  const Workspace w = workspace_layout(s);
+  AttnArgs a{};
+  a.s = s;
+  a.dense = 0;
+  a.row_ptr = idx->row_ptr;
+  a.cols = idx->cols;
+  a.route = idx->route;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.status = at<int>(ws, w.status);
+  a.trace = at<unsigned long long>(ws, w.trace);
+  a.scale_log2 = 0.12751743074380045f;  // log2(e) / sqrt(128)
+  a.qs = qs;
+  a.ks = ks;
+  CUtensorMap qm, km, vm;
+  rc = make_map3_u8(&qm, q8, (uint64_t)s.n, (uint64_t)s.h_q);
+  if (rc == CRISP_OK) rc = make_map3_u8(&km, k8, (uint64_t)s.n, (uint64_t)s.h_kv);
+  if (rc == CRISP_OK) rc = make_map3(&vm, v, (uint64_t)s.n, (uint64_t)s.h_kv, (uint64_t)s.ld);
+  if (rc != CRISP_OK) return rc;
+  return launch_sparse_attn(qm, km, vm, a, st) == cudaSuccess ? CRISP_OK : CRISP_ERR_CUDA;
+}
+
 int crisp_dense_prefill(const void* q, const void* k, const void* v, int h_q, int h_kv, int n, int d, void* o,
                         float* lse, void* ws, size_t ws_bytes, void* stream) {
   Shape s;

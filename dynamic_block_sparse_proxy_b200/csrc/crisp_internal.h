@@ -145,6 +145,10 @@ struct AttnArgs {
   int* status;
   unsigned long long* trace;
   float scale_log2;      // log2(e)/sqrt(d)
+  // FP8 logits (q_map and k_map then view E4M3 copies of Q and K): per (head, 128-row block)
+  // dequantisation scales [h_q][N_b] and [h_kv][N_b]; null for the bf16 kernel
+  const float* qs;
+  const float* ks;
 };
 
 // Launchers (return cudaGetLastError()).
@@ -156,6 +160,9 @@ cudaError_t launch_merge(const SelectArgs& a, cudaStream_t st);
 cudaError_t launch_sparse_attn(const CUtensorMap& q_map, const CUtensorMap& k_map,
                                const CUtensorMap& v_map, const AttnArgs& a, cudaStream_t st);
 cudaError_t launch_timeout_selftest(int* status, unsigned long long limit_ns, cudaStream_t st);
+// E4M3 copy [heads][n][128] of x (heads `ld` rows apart) and its per-block scales [heads][N_b].
+cudaError_t launch_fp8_quant(const __nv_bfloat16* x, int heads, int n, int ld, uint8_t* out, float* scales,
+                             cudaStream_t st);
 
 // SMs of the current device (queried once).
 int num_sms();

@@ -116,6 +116,9 @@ struct UnionWalk {
   }
 };
 
+// F8: Q and K arrive as E4M3 tiles (one 128x128-byte box each) and S = Q K^T runs as kind::f8f6f4
+// MMAs; the logit scale of a step folds in the two blocks' dequantisation scales.
+template <bool F8>
 __global__ void __launch_bounds__(THREADS, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap k_map,
                        const __grid_constant__ CUtensorMap v_map, const AttnArgs a) {
@@ -240,11 +243,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       tma_prefetch_desc(&q_map);
       tma_prefetch_desc(&k_map);
-      mbar_arrive_expect_tx(&sm.q_full, TILE_BYTES * ntiles);
+      mbar_arrive_expect_tx(&sm.q_full, (F8 ? HALF_BYTES : TILE_BYTES) * ntiles);
       for (int t = 0; t < ntiles; ++t) {
         const int qh = t ? tile_h[1] : tile_h[0], qy = (t ? tile_qb[1] : tile_qb[0]) * kB;
         tma_load_3d(&q_map, &sm.q_full, sm.q[t], 0, qy, qh);
-        tma_load_3d(&q_map, &sm.q_full, sm.q[t] + kB * 64, 64, qy, qh);
+        if (!F8) tma_load_3d(&q_map, &sm.q_full, sm.q[t] + kB * 64, 64, qy, qh);
       }
       UnionWalk u(tl, dense, tile_qb);
       int kb, mask, nk = 0;
@@ -254,9 +257,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int ky = kb * kB;
         trace_mark(a.trace, 0, 0, 1, step);
         if (!mbar_wait(&sm.k_empty[st], par, abort)) { fail(sm, a.status, CRISP_ERR_DEVICE_TIMEOUT); break; }
-        mbar_arrive_expect_tx(&sm.k_full[st], TILE_BYTES);
+        mbar_arrive_expect_tx(&sm.k_full[st], F8 ? HALF_BYTES : TILE_BYTES);
         tma_load_3d(&k_map, &sm.k_full[st], sm.k[st], 0, ky, kv);
-        tma_load_3d(&k_map, &sm.k_full[st], sm.k[st] + kB * 64, 64, ky, kv);
+        if (!F8) tma_load_3d(&k_map, &sm.k_full[st], sm.k[st] + kB * 64, 64, ky, kv);
         nk = step + 1;
       }
       if (u.bad) record_status(a.status, CRISP_ERR_DEVICE_CHECK);
@@ -348,10 +351,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (mask & bit) {
           tc_fence_after();
           const uint32_t ka = smem_u32(sm.k[st]);
+          if (F8) {
+            // E4M3 rows of 128 bytes: four MMAs of K = 32
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-            umma_ss(s_tmem, desc_kmajor_sw128(qa + off), desc_kmajor_sw128(ka + off), idesc_qk, kk > 0);
+            for (int kk = 0; kk < 4; ++kk)
+              umma_ss_f8(s_tmem, desc_kmajor_sw128(qa + kk * 32), desc_kmajor_sw128(ka + kk * 32),
+                         idesc_e4m3_f32(128, 128), kk > 0);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+              umma_ss(s_tmem, desc_kmajor_sw128(qa + off), desc_kmajor_sw128(ka + off), idesc_qk, kk > 0);
+            }
           }
           umma_commit(&sm.s_full[t]);
           umma_commit(&sm.k_empty[st]);
@@ -380,7 +391,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t lane_off = (uint32_t)(grp * 32) << 16;
     const uint32_t s_tmem = tmem + t * 128 + lane_off;
     const uint32_t o_tmem = tmem + 256 + t * 128 + lane_off;
-    const float sc = a.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     // Warp grp of tile 0 and warp grp of tile 1 share a sub-partition and its exp2 unit; they
@@ -410,6 +420,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         break;
       }
       tc_fence_after();
+      // the logit scale of this block (E4M3 logits: times both blocks' dequantisation scales)
+      const float sc = F8 ? a.scale_log2 * __ldg(a.qs + (size_t)my_h * s.nb + my_qb) * __ldg(a.ks + (size_t)kv * s.nb + kb)
+                          : a.scale_log2;
       // Exponentials use the row reference m of the earlier blocks without looking for this
       // block's maximum: fp32 (and bf16) share fp32's exponent range, so exp2(x*sc - m) stays
       // exact as long as it does not overflow. The first block sets m from its maximum; a later
@@ -544,11 +557,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 cudaError_t launch_sparse_attn(const CUtensorMap& q_map, const CUtensorMap& k_map, const CUtensorMap& v_map,
                                const AttnArgs& a, cudaStream_t st) {
   const size_t smem = sizeof(AttnSmem) + 1024;
-  cudaError_t e =
-      cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const bool f8 = a.qs != nullptr;
+  auto kernel = f8 ? sparse_attn_kernel<true> : sparse_attn_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int grid = a.s.h_q * ((a.s.nb + 1) / 2);
-  sparse_attn_kernel<<<grid, THREADS, smem, st>>>(q_map, k_map, v_map, a);
+  kernel<<<grid, THREADS, smem, st>>>(q_map, k_map, v_map, a);
   return cudaGetLastError();
 }
 

@@ -173,6 +173,31 @@ int crisp_dense_prefill(const void* q, const void* k, const void* v, int h_q, in
                         int d, void* o, float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * FP8 variant of the attention logits. The paper's pages quote an FP8 speedup only for another
+ * method (FlashPrefill V2); this is an optional variant, not the headline path. Q and K are first
+ * quantised to 8-bit E4M3 (the OCP 8-bit floating-point format: bias 7, 3 mantissa bits, largest
+ * finite value 448) per head and 128-row block: amax = max |x|, inv = 448 / amax and
+ * scale = amax / 448 (both rounded to fp32), code = E4M3(x * inv) with the product rounded to fp32
+ * and the value rounded to the nearest E4M3 (ties to even, saturating at 448); an all-zero block
+ * gets codes 0 and scale 1. The attention is then crisp_sparse_prefill's with S = Q K^T computed
+ * on the codes (tensor cores, fp32 accumulation) and each logit multiplied by the two blocks'
+ * scales: the exact attention of the dequantised Q and K up to the kernel's own rounding.
+ *
+ * crisp_fp8qk_buffer_size: bytes of the caller's buffer for the codes and scales, 0 for an
+ *   unsupported shape. Layout, each part starting on a 256-byte boundary, in this order:
+ *   Q codes uint8 [h_q][n][128], K codes uint8 [h_kv][n][128], Q scales float [h_q][N_b],
+ *   K scales float [h_kv][N_b].
+ * crisp_sparse_prefill_fp8qk: as crisp_sparse_prefill, plus fp8_buf (device, 256-byte aligned,
+ *   at least crisp_fp8qk_buffer_size bytes; overwritten, and left holding the codes and scales).
+ *   Errors as crisp_sparse_prefill; a missing or short buffer is CRISP_ERR_INVALID_ARG /
+ *   CRISP_ERR_WORKSPACE.
+ */
+size_t crisp_fp8qk_buffer_size(int h_q, int h_kv, int n, int d);
+int crisp_sparse_prefill_fp8qk(const void* q, const void* k, const void* v, int h_q, int h_kv, int n,
+                               int d, const crisp_index* idx, void* o, float* lse, void* ws,
+                               size_t ws_bytes, void* fp8_buf, size_t fp8_bytes, void* stream);
+
+/*
  * Synchronises `stream`, returns the device status word of `ws` (CRISP_OK or the first device
  * error recorded since the last call) and clears it. Returns CRISP_ERR_CUDA if the
  * synchronisation itself fails.

@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import dynamic_block_sparse_proxy_b200 as crisp
 from dynamic_block_sparse_proxy_b200 import build as B
@@ -199,3 +200,29 @@ def test_workspace_grows_with_length_including_partial_blocks(L):
     assert all(s > 0 and s % 256 == 0 for s in sizes)
     assert sizes == sorted(sizes)
     assert sizes[2] == L.crisp_workspace_size(4, 2, 128, 128, None) and sizes[3] > sizes[2]
+
+
+def test_fp8qk_buffer_size_and_argument_checks(L):
+    """The FP8 entry points: the buffer size follows the layout crisp.h documents (and the binding's
+    views mirror it), and a missing, misaligned or short buffer is refused before any launch."""
+    def layout(h_q, h_kv, n):
+        nb = -(-n // 128)
+        off = 0
+        for nbytes in (h_q * n * 128, h_kv * n * 128, h_q * nb * 4, h_kv * nb * 4):
+            off = -(-(off + nbytes) // 256) * 256
+        return off
+    for h_q, h_kv, n in ((32, 8, 131072), (28, 4, 3001), (1, 1, 1), (4, 2, 300)):
+        assert L.crisp_fp8qk_buffer_size(h_q, h_kv, n, 128) == layout(h_q, h_kv, n)
+    assert L.crisp_fp8qk_buffer_size(1, 1, 4096, 64) == 0
+    buf = torch.zeros(layout(4, 2, 300), dtype=torch.uint8)
+    q8, k8, qs, ks = crisp.fp8qk_views(buf, 4, 2, 300)
+    assert q8.shape == (4, 300, 128) and k8.shape == (2, 300, 128) and qs.shape == (4, 3) and ks.shape == (2, 3)
+    assert ks.data_ptr() + ks.numel() * 4 <= buf.data_ptr() + buf.numel()
+    fake, ws, big = 0x10000, 0x100000, 1 << 40
+    ix = _idx()
+    assert L.crisp_sparse_prefill_fp8qk(fake, fake, fake, 1, 1, 4096, 128, ctypes.byref(ix), fake, None, ws, big,
+                                        None, big, None) == -1
+    assert L.crisp_sparse_prefill_fp8qk(fake, fake, fake, 1, 1, 4096, 128, ctypes.byref(ix), fake, None, ws, big,
+                                        fake + 16, big, None) == -1
+    assert L.crisp_sparse_prefill_fp8qk(fake, fake, fake, 1, 1, 4096, 128, ctypes.byref(ix), fake, None, ws, big,
+                                        ws, 100, None) == -3
