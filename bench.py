@@ -138,12 +138,12 @@ def select_bytes(w, n_pe_heads: int, total_pairs: int) -> float:
 # (SHA-256 of the source, or of the selection sources in order); for any other source or workload
 # the bench reports null.
 ATTN_TRAFFIC = {"workload": "llama8b_128k",
-                "source_sha256": "93b54c6d7a93267e496f992d9f9bfeb5b74ee88130a05536d16d3d9c7ab6aecc",
-                "bytes": 2.70141e9 + 1.05458e9}
+                "source_sha256": "ba1487bcdca357eb7fce544ca872009ae1c3018bfa02d2e0dae827cb830a4843",
+                "bytes": 2.72104e9 + 1.05506e9}
 SELECT_SOURCES = ["proxy_pass.cu", "route_threshold.cu", "pe_cut.cu", "merge.cu", "sm100.cuh", "crisp_internal.h"]
 SELECT_TRAFFIC = {"workload": "llama8b_128k",
-                  "source_sha256": "e3c89aa9147e72fb8b5898aaaf057e16f3f2b5184f129b8756dd27bd55ae5b80",
-                  "bytes": 1283.68e6 + 88.04e6}
+                  "source_sha256": "134f564212b438969b5fb4cbf1ab7a41180d81fd7597859c5e87466119bcc3a3",
+                  "bytes": 1282.67e6 + 87.71e6}
 
 
 def _sources_sha(names):
