@@ -319,7 +319,7 @@ def run_crisp(args):
 
     e2e = None
     if args.e2e:
-        e2e = e2e_pipelined(w, q, k, v, params, idx, ws, max(4, min(args.steps, 8)), dev, stream)
+        e2e = e2e_pipelined(w, q, k, v, params, idx, ws, max(8, min(args.steps, 16)), dev, stream)
         e2e_s = max_over_ranks(e2e.pop("seconds_per_step"), world, dev)
         e2e.update(value=job_tokens_per_s(world, w.n, 1, e2e_s), ms_per_step=e2e_s * 1e3)
 
