@@ -185,12 +185,13 @@ def random_qkv(h_q: int, h_kv: int, n: int, d: int = 128, seed: int = 0, device=
 
 
 def spiked_qkv(h_q: int, h_kv: int, n: int, spike_blocks, gaps, d: int = 128, seed: int = 0, device="cpu",
-               q_rows=None):
+               q_rows=None, keys=(0, BLOCK)):
     """N(0,1) bf16 tensors with one planted direction u (|u|^2 = sqrt(d)): every key of the
     `spike_blocks` gets +w_k u and the queries of head h get +(gaps[h] / w_k) u, so that head's
     logits against the spiked keys rise by gaps[h] nats (q . k / sqrt(d) grows by w_q w_k).
-    `q_rows` limits the query term to a row range (e.g. the last 128 rows). Edge-case inputs for
-    the softmax reference handling: a spike far above the first key block a walk meets."""
+    `q_rows` limits the query term to a row range (e.g. the last 128 rows) and `keys` the spike to
+    a range of key offsets inside each spiked block. Edge-case inputs for the softmax reference
+    handling: a spike far above the first key block a walk meets."""
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
     q = torch.randn(h_q, n, d, generator=g)
@@ -199,7 +200,7 @@ def spiked_qkv(h_q: int, h_kv: int, n: int, spike_blocks, gaps, d: int = 128, se
     u = _planted_direction(g, d, "cpu")
     w_k = 8.0
     for kb in spike_blocks:
-        k[:, kb * BLOCK:min(n, (kb + 1) * BLOCK)] += w_k * u
+        k[:, min(n, kb * BLOCK + keys[0]):min(n, kb * BLOCK + keys[1])] += w_k * u
     lo, hi = q_rows if q_rows is not None else (0, n)
     for h in range(h_q):
         q[h, lo:hi] += (float(gaps[h]) / w_k) * u

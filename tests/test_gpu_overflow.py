@@ -101,6 +101,42 @@ def test_attention_redo_through_user_index(built, gap, hq, n, gaps_of):
     PT.assert_attention_ok(PT.compare_attention_blocks(q, k, v, o, lse, lists, blocks, hq))
 
 
+@pytest.mark.parametrize("keys", [(0, 64), (64, 128), (0, 16), (112, 128)])
+def test_half_block_spikes_pass_the_redo_threshold(keys):
+    """CPU check of the construction below: a spike on part of a block's keys alone lifts that
+    block's exponentials past the redo threshold against the first block."""
+    q, k, v = W.spiked_qkv(2, 1, 1024, [3, 6], [60.0, 100.0], seed=5, keys=keys)
+    _, k0, _ = W.spiked_qkv(2, 1, 1024, [3, 6], [60.0, 100.0], seed=5, keys=(0, 0))  # no spike
+    moved = (k.float() - k0.float()).abs().amax(dim=-1)[0]  # per key: touched by the spike?
+    for kb in (3, 6):
+        blk = moved[kb * 128:(kb + 1) * 128] > 0
+        assert blk[keys[0]:keys[1]].all() and blk.sum() == keys[1] - keys[0]
+    for h in range(2):
+        assert _gap_log2(q, k, h, 0, 0, 3, (512, 640)) > 64.0 + 8.0
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("keys", [(0, 64), (64, 128), (0, 16), (112, 128)])
+@pytest.mark.parametrize("hq,n", [(2, 1024), (1, 1000)])
+def test_attention_redo_by_key_range(built, keys, hq, n):
+    """The spike sits in only part of a block's keys (its first or its second 64 keys, or 16 of
+    them), at 60 and 100 nats, on a dense walk and a sparse one: the redo moves the reference
+    whichever keys carry the spike."""
+    q, k, v = W.spiked_qkv(hq, 1, n, [3, 6], [60.0, 100.0][:hq], seed=5, keys=keys)
+    q, k, v = q.to(dev()), k.to(dev()), v.to(dev())
+    nb = -(-n // 128)
+    lists = {h: _dense_lists(nb) for h in range(hq)}
+    lists[hq - 1] = [sorted({0, qb} | ({2, 3} if qb >= 3 else set()) | ({6} if qb >= 6 else set()))
+                     for qb in range(nb)]
+    idx = _index_from_lists([lists[h] for h in range(hq)], nb, [1] * hq)
+    ws = crisp.workspace(hq, 1, n, dev())
+    o, lse = crisp.sparse_prefill(q, k, v, idx, ws=ws)
+    crisp.check_status(ws)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+    blocks = [(h, qb) for h in range(hq) for qb in range(nb)]
+    PT.assert_attention_ok(PT.compare_attention_blocks(q, k, v, o, lse, lists, blocks, hq))
+
+
 @pytest.mark.gpu
 @pytest.mark.parametrize("gap", [60.0, 100.0])
 def test_dense_attention_redo(built, gap):
