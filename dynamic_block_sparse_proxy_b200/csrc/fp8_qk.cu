@@ -15,18 +15,25 @@
 namespace crisp {
 namespace {
 
-// One CTA per (head, 128-row block), thread t owns row t of the block (rows past n are skipped).
-__global__ void __launch_bounds__(kB) fp8_quant_kernel(const __nv_bfloat16* x, int n, int ld, int nb,
-                                                       uint8_t* out, float* scales) {
+constexpr int kQuantThreads = 256;
+constexpr int kChunks = kB * kD / 8;                 // 16-byte chunks of 8 values in a block
+constexpr int kPerThread = kChunks / kQuantThreads;  // 8
+
+// One CTA per (head, 128-row block). The block's rows are contiguous (kD values each), so thread
+// i takes the 16-byte chunks i, i + 256, ... of the block: every load and every 8-byte code store
+// of a warp covers one contiguous span. Chunk c holds row c / 16, values 8 (c % 16) .. +7; rows
+// past n are neither read nor stored.
+__global__ void __launch_bounds__(kQuantThreads) fp8_quant_kernel(const __nv_bfloat16* x, int n, int ld, int nb,
+                                                                  uint8_t* out, float* scales) {
   const int b = blockIdx.x, h = blockIdx.y, t = threadIdx.x;
-  const int row = b * kB + t;
-  const bool live = row < n;
-  const uint4* src = reinterpret_cast<const uint4*>(x + ((size_t)h * ld + (live ? row : 0)) * kD);
-  uint4 u[kD / 8];
+  const int rows = min(kB, n - b * kB);  // rows of this block below n
+  const uint4* src = reinterpret_cast<const uint4*>(x + ((size_t)h * ld + (size_t)b * kB) * kD);
+  uint4 u[kPerThread];
   float amax = 0.f;
 #pragma unroll
-  for (int i = 0; i < kD / 8; ++i) {
-    u[i] = live ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+  for (int i = 0; i < kPerThread; ++i) {
+    const int c = t + i * kQuantThreads;
+    u[i] = c / (kD / 8) < rows ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
     const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&u[i]);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -36,30 +43,32 @@ __global__ void __launch_bounds__(kB) fp8_quant_kernel(const __nv_bfloat16* x, i
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  __shared__ float wmax[kB / 32];
+  __shared__ float wmax[kQuantThreads / 32];
   if ((t & 31) == 0) wmax[t >> 5] = amax;
   __syncthreads();
-  amax = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
+  amax = wmax[0];
+#pragma unroll
+  for (int w = 1; w < kQuantThreads / 32; ++w) amax = fmaxf(amax, wmax[w]);
   const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
   if (t == 0) scales[(size_t)h * nb + b] = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
-  if (!live) return;
-  uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)h * n + row) * kD);  // n rows per head
+  uint2* dst = reinterpret_cast<uint2*>(out + ((size_t)h * n + (size_t)b * kB) * kD);  // n rows per head
 #pragma unroll
-  for (int i = 0; i < kD / 16; ++i) {
-    uint32_t w[4];
+  for (int i = 0; i < kPerThread; ++i) {
+    const int c = t + i * kQuantThreads;
+    if (c / (kD / 8) >= rows) continue;
+    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&u[i]);
+    uint32_t w[2];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      // 4 values: bf16 pairs 2j and 2j+1 of the 16 in u[2i], u[2i+1]
-      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&u[2 * i + (j >> 1)]);
-      const float2 f0 = __bfloat1622float2(p2[(j & 1) * 2]);
-      const float2 f1 = __bfloat1622float2(p2[(j & 1) * 2 + 1]);
+    for (int j = 0; j < 2; ++j) {
+      const float2 f0 = __bfloat1622float2(p2[2 * j]);
+      const float2 f1 = __bfloat1622float2(p2[2 * j + 1]);
       const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(__fmul_rn(f0.x, inv), __fmul_rn(f0.y, inv)),
                                                               __NV_SATFINITE, __NV_E4M3);
       const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(make_float2(__fmul_rn(f1.x, inv), __fmul_rn(f1.y, inv)),
                                                               __NV_SATFINITE, __NV_E4M3);
       w[j] = (uint32_t)lo | ((uint32_t)hi << 16);
     }
-    dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+    dst[c] = make_uint2(w[0], w[1]);
   }
 }
 
@@ -68,7 +77,7 @@ __global__ void __launch_bounds__(kB) fp8_quant_kernel(const __nv_bfloat16* x, i
 cudaError_t launch_fp8_quant(const __nv_bfloat16* x, int heads, int n, int ld, uint8_t* out, float* scales,
                              cudaStream_t st) {
   const int nb = (n + kB - 1) / kB;
-  fp8_quant_kernel<<<dim3(nb, heads), kB, 0, st>>>(x, n, ld, nb, out, scales);
+  fp8_quant_kernel<<<dim3(nb, heads), kQuantThreads, 0, st>>>(x, n, ld, nb, out, scales);
   return cudaGetLastError();
 }
 
