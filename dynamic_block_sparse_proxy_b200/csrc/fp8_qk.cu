@@ -51,6 +51,7 @@ __global__ void __launch_bounds__(kQuantThreads) fp8_quant_kernel(const __nv_bfl
   for (int w = 1; w < kQuantThreads / 32; ++w) amax = fmaxf(amax, wmax[w]);
   const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
   if (t == 0) scales[(size_t)h * nb + b] = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+  const uint32_t keep = amax > 0.f ? 0xffffffffu : 0u;  // an all-zero block (signed zeros too): codes 0
   uint2* dst = reinterpret_cast<uint2*>(out + ((size_t)h * n + (size_t)b * kB) * kD);  // n rows per head
 #pragma unroll
   for (int i = 0; i < kPerThread; ++i) {
@@ -68,7 +69,7 @@ __global__ void __launch_bounds__(kQuantThreads) fp8_quant_kernel(const __nv_bfl
                                                               __NV_SATFINITE, __NV_E4M3);
       w[j] = (uint32_t)lo | ((uint32_t)hi << 16);
     }
-    dst[c] = make_uint2(w[0], w[1]);
+    dst[c] = make_uint2(w[0] & keep, w[1] & keep);
   }
 }
 

@@ -63,6 +63,48 @@ def test_fp8_codes_and_scales_bit_exact(built, name, n):
         assert np.array_equal(scales.cpu().numpy(), osc), (name, n)
 
 
+def _edge_blocks() -> torch.Tensor:
+    """Two heads of 640 rows whose blocks reach the quantiser's special cases: all zeros, all
+    negative zeros (scale 1 and codes 0 either way), one large value beside values a million times
+    smaller (subnormal and zero codes), and a block whose maximum is exactly 448, so that values
+    pass unscaled and those halfway between E4M3 neighbours, subnormal and normal, positive and
+    negative, are settled by the ties-to-even rule."""
+    n, d = 640, 128
+    g = torch.Generator().manual_seed(3)
+    x = torch.randn(2, n, d, generator=g)
+    x[0, 0:128] = 0.0
+    x[0, 128:256] = -0.0
+    x[0, 256:384] *= 1e-3
+    x[0, 300, 5] = 1e3
+    t = torch.zeros(128, d)
+    t[0, 0] = 448.0
+    halfway = [(m + 0.5) * 2.0 ** -9 for m in range(8)] + [1.0625, 1.1875, 17.0, 19.0, 104.0, 0.0146484375]
+    for i, val in enumerate(halfway):
+        t[1 + i, :] = val
+        t[40 + i, :] = -val
+    x[1, 128:256] = t
+    return x.to(torch.bfloat16)
+
+
+def test_fp8_codes_edge_blocks_bit_exact(built):
+    q = _edge_blocks()
+    k = _edge_blocks()[:1].flip(1).contiguous()
+    v = torch.randn(1, q.shape[1], 128, generator=torch.Generator().manual_seed(4)).to(torch.bfloat16)
+    qd, kd, vd = q.to(dev()), k.to(dev()), v.to(dev())
+    ws = crisp.workspace(2, 1, q.shape[1], dev())
+    idx = crisp.select(qd, kd, crisp.Params(), ws=ws)
+    o, lse, buf = crisp.sparse_prefill_fp8qk(qd, kd, vd, idx, ws=ws)
+    crisp.check_status(ws)
+    q8, k8, qs, ks = crisp.fp8qk_views(buf, 2, 1, q.shape[1])
+    for x, codes, scales in ((q, q8, qs), (k, k8, ks)):
+        _, oc, osc = _dequantised(x)
+        gc = codes.cpu().numpy()
+        bad = np.nonzero(gc != oc)
+        assert bad[0].size == 0, (bad[0][:5], bad[1][:5], bad[2][:5], gc[bad][:5], oc[bad][:5])
+        assert np.array_equal(scales.cpu().numpy(), osc)
+    assert torch.isfinite(o.float()).all()
+
+
 @pytest.mark.parametrize("name,n", [("tiny_1h_4k", 4096), ("llama8b_32k", 8192), ("llama8b_32k", 3001)])
 def test_fp8_attention_matches_dequantised_oracle(built, name, n):
     w = W.WORKLOADS[name].scaled(-(-n // 128) * 128)
