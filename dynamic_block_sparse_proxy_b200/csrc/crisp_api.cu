@@ -2,6 +2,7 @@
 // encoding and the launch sequence of each entry point. Nothing here allocates device memory;
 // every buffer comes from the caller.
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cmath>
 #include <cstring>
@@ -11,6 +12,16 @@
 
 namespace crisp {
 namespace {
+
+// NVTX push/pop range over a scope: the kernels launched inside it carry the range's name in a
+// profiler (ncu --nvtx --nvtx-include "crisp_select/" selects the selection kernels). With no
+// profiler attached a push or pop is a call through a no-op pointer.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   // Resolved once through the runtime (no link-time dependency on libcuda).
@@ -100,6 +111,7 @@ T* at(void* ws, size_t off) {
 
 int run_select(const void* q, const void* k, const Shape& s, const crisp_params* p, const crisp_index& out,
                void* ws, int* status, cudaStream_t st) {
+  NvtxRange range("crisp_select");
   const Workspace w = workspace_layout(s);
   SelectArgs a{};
   a.s = s;
@@ -155,10 +167,22 @@ int run_select(const void* q, const void* k, const Shape& s, const crisp_params*
   // from zero (the arrays are contiguous).
   if (cudaMemsetAsync(at<uint8_t>(ws, w.hist_cnt), 0, w.cut_done + (size_t)s.h_q * 4 - w.hist_cnt, st) != cudaSuccess)
     return CRISP_ERR_CUDA;
-  if (launch_proxy_pass(qm, km, a, st) != cudaSuccess) return CRISP_ERR_CUDA;
-  if (launch_route_threshold(a, st) != cudaSuccess) return CRISP_ERR_CUDA;
-  if (launch_pe(a, qpm, kpm, st) != cudaSuccess) return CRISP_ERR_CUDA;
-  if (launch_merge(a, st) != cudaSuccess) return CRISP_ERR_CUDA;
+  {
+    NvtxRange stage("proxy_pass");
+    if (launch_proxy_pass(qm, km, a, st) != cudaSuccess) return CRISP_ERR_CUDA;
+  }
+  {
+    NvtxRange stage("route_threshold");
+    if (launch_route_threshold(a, st) != cudaSuccess) return CRISP_ERR_CUDA;
+  }
+  {
+    NvtxRange stage("pooled_estimation");
+    if (launch_pe(a, qpm, kpm, st) != cudaSuccess) return CRISP_ERR_CUDA;
+  }
+  {
+    NvtxRange stage("merge");
+    if (launch_merge(a, st) != cudaSuccess) return CRISP_ERR_CUDA;
+  }
   return CRISP_OK;
 }
 
@@ -184,6 +208,7 @@ int run_attention(const void* q, const void* k, const void* v, const Shape& s, c
   if (rc == CRISP_OK) rc = make_map3(&km, k, (uint64_t)s.n, (uint64_t)s.h_kv, (uint64_t)s.ld);
   if (rc == CRISP_OK) rc = make_map3(&vm, v, (uint64_t)s.n, (uint64_t)s.h_kv, (uint64_t)s.ld);
   if (rc != CRISP_OK) return rc;
+  NvtxRange range(dense ? "crisp_dense_attention" : "crisp_attention");
   return launch_sparse_attn(qm, km, vm, a, st) == cudaSuccess ? CRISP_OK : CRISP_ERR_CUDA;
 }
 
@@ -392,9 +417,12 @@ int crisp_sparse_prefill_fp8qk(const void* q, const void* k, const void* v, int 
   uint8_t* k8 = at<uint8_t>(fp8_buf, f.k8);
   float* qs = at<float>(fp8_buf, f.qs);
   float* ks = at<float>(fp8_buf, f.ks);
-  if (launch_fp8_quant(static_cast<const __nv_bfloat16*>(q), s.h_q, s.n, s.ld, q8, qs, st) != cudaSuccess ||
-      launch_fp8_quant(static_cast<const __nv_bfloat16*>(k), s.h_kv, s.n, s.ld, k8, ks, st) != cudaSuccess)
-    return CRISP_ERR_CUDA;
+  {
+    NvtxRange range("crisp_fp8_quantise");
+    if (launch_fp8_quant(static_cast<const __nv_bfloat16*>(q), s.h_q, s.n, s.ld, q8, qs, st) != cudaSuccess ||
+        launch_fp8_quant(static_cast<const __nv_bfloat16*>(k), s.h_kv, s.n, s.ld, k8, ks, st) != cudaSuccess)
+      return CRISP_ERR_CUDA;
+  }
   const Workspace w = workspace_layout(s);
   AttnArgs a{};
   a.s = s;
@@ -414,6 +442,7 @@ int crisp_sparse_prefill_fp8qk(const void* q, const void* k, const void* v, int 
   if (rc == CRISP_OK) rc = make_map3_u8(&km, k8, (uint64_t)s.n, (uint64_t)s.h_kv);
   if (rc == CRISP_OK) rc = make_map3(&vm, v, (uint64_t)s.n, (uint64_t)s.h_kv, (uint64_t)s.ld);
   if (rc != CRISP_OK) return rc;
+  NvtxRange range("crisp_attention_fp8qk");
   return launch_sparse_attn(qm, km, vm, a, st) == cudaSuccess ? CRISP_OK : CRISP_ERR_CUDA;
 }
 

@@ -27,6 +27,12 @@
  *   - The workspace's first 256 bytes hold the device status word: zero them once after
  *     allocating the workspace (e.g. cudaMemset); crisp_get_status() clears it after reading.
  *     The rest of the workspace needs no initialisation and may hold anything between calls.
+ *   - Tracing: the launches sit inside NVTX push/pop ranges named "crisp_select" (with
+ *     "proxy_pass", "route_threshold", "pooled_estimation" and "merge" nested in it),
+ *     "crisp_attention", "crisp_dense_attention", "crisp_fp8_quantise" and
+ *     "crisp_attention_fp8qk", so a profiler can pick a stage's kernels (for example
+ *     ncu --nvtx --nvtx-include "crisp_select/"). Without a profiler attached they cost a call
+ *     through a no-op pointer.
  */
 #ifndef CRISP_H
 #define CRISP_H
