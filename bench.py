@@ -102,9 +102,16 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.f.close()
+        with open(self.path) as f:
+            return self.summarise(f)
+
+    @staticmethod
+    def summarise(lines) -> dict:
+        """Median SM clock, the maximum clock and the throttle reasons seen active, from
+        `nvidia-smi --query-gpu=<QUERY> --format=csv,noheader,nounits` lines."""
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
+        for line in lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
