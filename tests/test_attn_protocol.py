@@ -22,34 +22,16 @@ import random
 
 import pytest
 
+from tests.protocol_sim import Bar, Sim
+
 NSK, NSV = 2, 3
 
 
-class Bar:
-    def __init__(self, name, count):
-        self.name, self.count, self.pending, self.phase = name, count, count, 0
-
-    def arrive(self):
-        self.pending -= 1
-        assert self.pending >= 0, self.name
-        if self.pending == 0:
-            self.phase += 1
-            self.pending = self.count
-
-    def done(self, k):
-        """Has phase k (0-based) completed? The kernel tests parity k & 1, which is only sound
-        while the barrier is at most one phase past k."""
-        assert self.phase <= k + 1, (f"{self.name}: phase {self.phase} while phase {k} is awaited "
-                                     "(a parity wait would alias)")
-        return self.phase > k
-
-
-class Model:
+class Model(Sim):
     def __init__(self, masks, ntiles, seed, broken=None):
-        self.rng = random.Random(seed)
+        super().__init__(seed)
         self.broken = broken  # a deliberate protocol mistake, for the tests that pin the model
         self.masks, self.ntiles = masks, ntiles
-        self.events, self.time = [], 0
         self.q_full = Bar("q_full", 1)
         self.k_full = [Bar(f"k_full{i}", 1) for i in range(NSK)]
         self.k_empty = [Bar(f"k_empty{i}", ntiles) for i in range(NSK)]
@@ -66,9 +48,6 @@ class Model:
         self.s_reads = [0, 0]  # blocks whose S the softmax has read
         self.pv_done = [0, 0]  # PVs completed
         self.tail = [0, 0]  # completion time of each issuer's last MMA
-
-    def later(self, delay, fn):
-        self.events.append((self.time + delay, fn))
 
     # ---------------------------------------------------------------- asynchronous units
     def fill(self, slots, full, st, step):
@@ -199,43 +178,12 @@ class Model:
             i += 1
         yield (self.o_done[t], 0)
 
-    # ---------------------------------------------------------------- scheduler
-    def pop_event(self):
-        self.events.sort(key=lambda e: e[0])
-        tm, fn = self.events.pop(0)
-        self.time = max(self.time, tm)
-        fn()
-
-    def run(self):
+    def roles(self):
         roles = {"kp": self.k_producer(), "vp": self.v_producer()}
         for t in range(self.ntiles):
             roles[f"mma{t}"] = self.issuer(t)
             roles[f"softmax{t}"] = self.softmax(t)
-        blocked = {name: None for name in roles}
-        finished = set()
-        for _ in range(10 ** 6):
-            if len(finished) == len(roles):
-                break
-            runnable = [r for r in roles if r not in finished and (blocked[r] is None or blocked[r][0].done(blocked[r][1]))]
-            if not runnable or (self.events and self.rng.random() < 0.3):
-                if not self.events:
-                    waits = ", ".join(f"{r} on {b[0].name} phase {b[1]}" for r, b in blocked.items()
-                                      if r not in finished and b)
-                    raise AssertionError("deadlock: " + waits)
-                self.pop_event()
-                continue
-            r = self.rng.choice(runnable)
-            blocked[r] = None
-            try:
-                w = next(roles[r])
-                if w is not None and not w[0].done(w[1]):
-                    blocked[r] = w
-            except StopIteration:
-                finished.add(r)
-        else:
-            raise AssertionError("no progress")
-        while self.events:
-            self.pop_event()
+        return roles
 
 
 def random_masks(rng, L, ntiles):
